@@ -1,0 +1,443 @@
+#!/usr/bin/env python
+"""Decode throughput of the ARKV tri-state KV-cache path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl arkv|reference]
+
+A step is one decode step of the whole attention stack: for every layer, append +
+mixed-precision attention (arkv_decode_attn), score update (arkv_score_update),
+and the tier reassignment (arkv_reassign) on every reassign_interval-th step.
+Each GPU runs its own replica of the workload (independent sequences; no
+collective on the data path), so `value` is the tokens/s of all ranks together
+("scaling": "weak").  Inputs are synthetic and seeded; each step streams the whole
+compressed cache (GBs, far above the 126 MB L2), so no L2 flush is needed.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixed_precision_kv_arkv_b200 import workloads  # noqa: E402
+
+METRIC = "decode tokens/s & HBM GB/s (% of peak), tri-state KV attention, 8B shape 32K"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=128)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=workloads.LLAMA3_8B.name, choices=sorted(workloads.BY_NAME))
+    ap.add_argument("--impl", default="arkv", choices=["arkv", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_traffic(kernel_file: str):
+    """DRAM bytes per launch of the decode kernel from the committed ncu summary, if
+    it was taken on the current kernel source (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "decode_attn_traffic.txt")
+    src = os.path.join(ROOT, "mixed_precision_kv_arkv_b200", "csrc", kernel_file)
+    try:
+        kv = dict(line.split(":", 1) for line in open(path) if ":" in line)
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if kv.get("kernel_src_sha256_16", "").strip() != sha:
+            return None
+        return float(kv["dram_bytes_per_launch_scaled"].strip())
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local_rank: int):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        self.index = ids[local_rank] if local_rank < len(ids) else str(local_rank)
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.first = self.proc.stdout.readline()     # sampling has started
+        except Exception:
+            self.proc = None
+            self.first = ""
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.out = self.out or ""
+        return False
+
+    def summary(self):
+        rows = [r for r in csv.reader(io.StringIO(self.out or "")) if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ CPU baseline (the oracle)
+class OracleSampler:
+    """The oracle on a bounded sample of the workload: some rows of layer 0, set up
+    once (prefill + initial reassignment, untimed), then timed decode steps
+    (attention + score update, and the reassignment on its steps)."""
+
+    def __init__(self, wl, rows=(0,)):
+        from threadpoolctl import threadpool_info
+        from mixed_precision_kv_arkv_b200 import inputs
+        from oracle import arkv as A
+
+        self.wl, self.rows, self.inputs = wl, list(rows), inputs
+        pre = inputs.layer_prefill(wl, 0, 0, seqs=sorted({r // wl.hkv for r in rows}),
+                                   kv_heads=sorted({r % wl.hkv for r in rows}))
+        f = inputs.bf16_to_f64
+        self.lay = A.OracleLayer(wl.batch, wl.hq, wl.hkv, wl.head_dim, wl.window, wl.n_obs,
+                                 wl.budget_frac, wl.gamma, pre["ctx_len"], rows=self.rows)
+        self.lay.prefill(f(pre["k"]), f(pre["v"]), f(pre["q_obs"]))
+        self.r = wl.oq_ratio if wl.oq_ratio is not None else wl.r_bar
+        self.lay.initial_reassign(self.r)
+        self.t = 0
+        self.threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+
+    def step(self) -> float:
+        """One timed decode step of the sampled rows; seconds per row-step."""
+        wl, f = self.wl, self.inputs.bf16_to_f64
+        d = self.inputs.decode_inputs(wl, 0, self.t)
+        t0 = time.perf_counter()
+        self.lay.decode_step(self.t, f(d["q"]), f(d["k_new"]), f(d["v_new"]))
+        if (self.t + 1) % wl.reassign_interval == 0:
+            self.lay.reassign(self.t, self.r)
+        dt = time.perf_counter() - t0
+        self.t += 1
+        return dt / len(self.rows)
+
+    def describe(self, n_steps):
+        wl = self.wl
+        return (f"oracle on row(s) {self.rows} of layer 0 ({wl.name}), {n_steps} decode steps "
+                f"incl. reassignments every {wl.reassign_interval}; time per row-step scaled to "
+                f"{wl.layers} layers x {wl.rows} rows")
+
+
+def cpu_baseline_line(wl, seconds):
+    smp = OracleSampler(wl)
+    per, spent = [], 0.0
+    while len(per) < wl.reassign_interval or spent < seconds:
+        per.append(smp.step())
+        spent += per[-1] * len(smp.rows)
+    step_s = statistics.mean(per) * wl.rows * wl.layers
+    return {"value": wl.batch / step_s, "unit": "tokens/s", "cores": smp.threads, "kind": "oracle",
+            "sample": smp.describe(len(per))}
+
+
+def run_reference(args, wl, rank):
+    if rank != 0:
+        return
+    smp = OracleSampler(wl)
+    per = []
+    for i in range(args.warmup + args.steps):
+        x = smp.step()
+        if i >= args.warmup:
+            per.append(x)
+    step_s = statistics.mean(per) * wl.rows * wl.layers
+    value = wl.batch / step_s
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(wl),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": smp.threads,
+                             "kind": "oracle", "sample": smp.describe(len(per))},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(wl):
+    return {"workload": wl.name, "layers": wl.layers, "batch": wl.batch, "hq": wl.hq, "hkv": wl.hkv,
+            "head_dim": wl.head_dim, "n_ctx": wl.n_ctx, "n_ctx_min": wl.n_ctx_min,
+            "budget_frac": wl.budget_frac, "oq_ratio": wl.oq_ratio if wl.oq_ratio is not None
+            else f"per layer from prefill stats (r_bar {wl.r_bar})", "window": wl.window,
+            "gamma": wl.gamma, "reassign_interval": wl.reassign_interval,
+            "l2": "no flush: every step streams the whole compressed cache, far above L2"}
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_arkv(args, wl, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from mixed_precision_kv_arkv_b200 import abi, build, inputs
+    from mixed_precision_kv_arkv_b200.cache import LayerCache, Workspace, make_cfg, stream_ptr
+
+    build.build()
+    abi.lib()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    s = stream_ptr()
+    L, B, Hq, Hkv, D = wl.layers, wl.batch, wl.hq, wl.hkv, wl.head_dim
+    K, W = args.steps, args.warmup
+    passes = 1 + (0 if args.no_e2e else 1) + 1          # value, e2e, kernel timing
+    total_steps = W + passes * K
+    ctx_np = inputs.ctx_lengths(wl, 0)
+    n_max = int(ctx_np.max()) + total_steps
+    ctx = torch.from_numpy(ctx_np).to(dev)
+
+    # ---------- prefill statistics of every layer, then the per-layer Original share
+    probe = make_cfg(B, Hq, Hkv, D, wl.window, wl.n_obs, wl.gamma, wl.budget_frac, 1, 1)
+    ws_pre = Workspace(abi.arkv_workspace_bytes(probe, abi.ARKV_WS_PREFILL, wl.n_ctx), dev)
+    stats = torch.zeros((L, 3), dtype=torch.float64, device=dev)
+    mu0 = torch.zeros((wl.rows, wl.n_ctx), dtype=torch.float32, device=dev)
+    m20 = torch.zeros_like(mu0)
+    seed = rank
+    for l in range(L):
+        pre = inputs.layer_prefill_torch(wl, l, dev, seed, ctx_np)
+        abi.arkv_prefill_stats(probe, pre["q_obs"].data_ptr(), pre["k"].data_ptr(), wl.n_ctx,
+                               ctx.data_ptr(), stats[l].data_ptr(), None, mu0.data_ptr(),
+                               m20.data_ptr(), ws_pre.ptr, ws_pre.nbytes, s)
+        del pre
+    st_host = stats.cpu().numpy()
+    if wl.oq_ratio is not None:
+        r = np.full(L, wl.oq_ratio, np.float32)
+    else:
+        r = np.zeros(L, np.float32)
+        abi.arkv_oq_ratio(st_host.ctypes.data, L, wl.r_bar, r.ctypes.data)
+
+    # ---------- per-layer caches: capacities, initial pack
+    layers = []
+    for l in range(L):
+        cap_o, cap_q = abi.arkv_row_capacity(probe, n_max, float(r[l]), wl.reassign_interval)
+        cfg = make_cfg(B, Hq, Hkv, D, wl.window, wl.n_obs, wl.gamma, wl.budget_frac, cap_o, cap_q)
+        cache = LayerCache(cfg, dev)
+        pre = inputs.layer_prefill_torch(wl, l, dev, seed, ctx_np)
+        abi.arkv_prefill_stats(cfg, pre["q_obs"].data_ptr(), pre["k"].data_ptr(), wl.n_ctx,
+                               ctx.data_ptr(), stats[l].data_ptr(), None, mu0.data_ptr(),
+                               m20.data_ptr(), ws_pre.ptr, ws_pre.nbytes, s)
+        abi.arkv_quantize_pack(cfg, float(r[l]), pre["k"].data_ptr(), pre["v"].data_ptr(), wl.n_ctx,
+                               ctx.data_ptr(), mu0.data_ptr(), m20.data_ptr(), cache.c, None,
+                               ws_pre.ptr, ws_pre.nbytes, s)
+        dec = inputs.decode_inputs_torch(wl, pre["u"], total_steps, dev, seed, l)
+        layers.append({"cfg": cfg, "cache": cache, "r": float(r[l]), "dec": dec,
+                       "ws_d": Workspace(abi.arkv_workspace_bytes(cfg, abi.ARKV_WS_DECODE), dev),
+                       "ws_r": Workspace(abi.arkv_workspace_bytes(cfg, abi.ARKV_WS_REASSIGN), dev)})
+        del pre
+    del ws_pre, mu0, m20
+    torch.cuda.synchronize()
+    status = sum(int(x["cache"].status.item()) for x in layers)
+    assert status == 0, f"cache status {status} after pack"
+    o = torch.zeros((L, B, Hq, D), dtype=torch.float32, device=dev)
+    launches = {"n": 0}
+
+    def layer_step(l, t, q=None, kn=None, vn=None, ev=None):
+        x = layers[l]
+        cfg, c = x["cfg"], x["cache"].c
+        q = x["dec"]["q"][t] if q is None else q
+        kn = x["dec"]["k_new"][t] if kn is None else kn
+        vn = x["dec"]["v_new"][t] if vn is None else vn
+        if ev is not None:
+            ev[0].record()
+        abi.arkv_decode_attn(cfg, t, q.data_ptr(), kn.data_ptr(), vn.data_ptr(), ctx.data_ptr(), c,
+                             o[l].data_ptr(), x["ws_d"].ptr, x["ws_d"].nbytes, stream_ptr())
+        if ev is not None:
+            ev[1].record()
+        abi.arkv_score_update(cfg, t, ctx.data_ptr(), c, x["ws_d"].ptr, x["ws_d"].nbytes, stream_ptr())
+        launches["n"] += 2
+        if (t + 1) % wl.reassign_interval == 0:
+            abi.arkv_reassign(cfg, t, x["r"], ctx.data_ptr(), c, None, x["ws_r"].ptr, x["ws_r"].nbytes,
+                              stream_ptr())
+            launches["n"] += 1
+
+    for t in range(W):                                       # warm-up, eager
+        for l in range(L):
+            layer_step(l, t)
+    torch.cuda.synchronize()
+
+    def capture(t0, nsteps, body):
+        graphs, t = [], t0
+        while t < t0 + nsteps:
+            n = min(wl.reassign_interval - (t % wl.reassign_interval), t0 + nsteps - t)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for tt in range(t, t + n):
+                    body(tt)
+            graphs.append(g)
+            t += n
+        return graphs
+
+    # ---------- pass 1: device-timed value
+    t_value = W
+    g_value = capture(t_value, K, lambda tt: [layer_step(l, tt) for l in range(L)])
+    launches["n"] = 0
+    for tt in range(t_value, t_value + K):
+        for l in range(L):
+            launches["n"] += 2 + (1 if (tt + 1) % wl.reassign_interval == 0 else 0)
+    gpu_launches = launches["n"]
+
+    # ---------- pass 2: end to end through host buffers
+    t_e2e = W + K
+    h2d = d2h = 0
+    if not args.no_e2e:
+        qh = torch.stack([x["dec"]["q"][t_e2e:t_e2e + K] for x in layers], 1).cpu().pin_memory()
+        kh = torch.stack([x["dec"]["k_new"][t_e2e:t_e2e + K] for x in layers], 1).cpu().pin_memory()
+        vh = torch.stack([x["dec"]["v_new"][t_e2e:t_e2e + K] for x in layers], 1).cpu().pin_memory()
+        oh = torch.empty((K, L, B, Hq, D), dtype=torch.float32).pin_memory()
+        qd, kd, vd = (torch.empty_like(qh[0], device=dev), torch.empty_like(kh[0], device=dev),
+                      torch.empty_like(vh[0], device=dev))
+        h2d = qh[0].numel() * 2 + kh[0].numel() * 2 + vh[0].numel() * 2
+        d2h = oh[0].numel() * 4
+
+        def e2e_body(tt):
+            i = tt - t_e2e
+            qd.copy_(qh[i], non_blocking=True)
+            kd.copy_(kh[i], non_blocking=True)
+            vd.copy_(vh[i], non_blocking=True)
+            for l in range(L):
+                layer_step(l, tt, qd[l], kd[l], vd[l])
+            oh[i].copy_(o, non_blocking=True)
+        g_e2e = capture(t_e2e, K, e2e_body)
+
+    # ---------- pass 3: the decode kernel timed by events on its stream
+    t_k = W + (passes - 1) * K
+    evs = [(torch.cuda.Event(enable_timing=True, external=True),
+            torch.cuda.Event(enable_timing=True, external=True)) for _ in range(K * L)]
+    counts = torch.zeros((K, L, 2, wl.rows), dtype=torch.int32, device=dev)
+
+    def k_body(tt):
+        i = tt - t_k
+        for l in range(L):
+            counts[i, l, 0].copy_(layers[l]["cache"].n_bf16)
+            counts[i, l, 1].copy_(layers[l]["cache"].n_fp8)
+            layer_step(l, tt, ev=evs[i * L + l])
+    g_k = capture(t_k, K, k_body)
+
+    def timed(graphs):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for g in graphs:
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b)
+        if world > 1:
+            tm = torch.tensor([ms], device=dev)
+            dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+            ms = float(tm.item())
+        return ms
+
+    with ClockSampler(local_rank) as clk:
+        ms_value = timed(g_value)
+        ms_e2e = timed(g_e2e) if not args.no_e2e else None
+        timed(g_k)
+    clocks = clk.summary()
+    clocks["window"] = "sampled every 50 ms across the three timed passes"
+    k1_ms = [a.elapsed_time(b) for a, b in evs]
+    cn = counts.cpu().numpy().astype(np.int64)               # [K, L, 2, rows] before each launch
+    per_row = (cn[:, :, 0] + 1) * 4 * D + cn[:, :, 1] * (2 * D + 8)
+    io_bytes = B * Hq * D * 2 + B * Hq * D * 4 + 2 * B * Hkv * D * 2
+    alg_bytes = per_row.sum(-1) + io_bytes                   # [K, L]
+    achieved = float(alg_bytes.sum() / (sum(k1_ms) * 1e-3) / 1e9)
+    peak, peak_kind = hbm_peak()
+    step_bytes = float(alg_bytes.sum(-1).mean())
+
+    status = sum(int(x["cache"].status.item()) for x in layers)
+    tokens = B * K * world
+    value = tokens / (ms_value * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": ms_value / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_of(wl),
+        "hbm_gbs_step": step_bytes / (ms_value / K * 1e-3) / 1e9,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": kernel_traffic("decode_attn.cu"),
+                     "kernel": "decode_attn_kernel<128>" if D == 128 else "decode_attn_kernel<64>",
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                     else "fallback 6650 GB/s",
+                     "bytes_per_launch": float(alg_bytes.mean()),
+                     "ms_per_launch": statistics.mean(k1_ms)},
+        "gpu_launches": gpu_launches,
+        "clocks": clocks,
+        "oq_ratio_per_layer": [round(float(x), 4) for x in r],
+        "cache_status": status,
+    }
+    if not args.no_e2e:
+        line["e2e"] = {"value": tokens / (ms_e2e * 1e-3), "unit": "tokens/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "ms_per_step": ms_e2e / K}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_line(wl, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del g_value, g_k
+    if not args.no_e2e:
+        del g_e2e
+
+
+def main():
+    args = parse()
+    wl = workloads.BY_NAME[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, wl, rank)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_arkv(args, wl, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
