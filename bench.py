@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="run only this many layers of the workload (profiling a smaller case)")
     return ap.parse_args()
 
 
@@ -418,6 +420,8 @@ def run_arkv(args, wl, rank, world, local_rank):
 def main():
     args = parse()
     wl = workloads.BY_NAME[args.workload]
+    if args.layers is not None:
+        wl = wl.with_(layers=args.layers)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
