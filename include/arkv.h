@@ -199,6 +199,25 @@ int arkv_reassign(const arkv_cfg *cfg, int32_t step, float r, const int32_t *ctx
  * even, saturate to +-448), for testing: out[i] = code(x[i]), n elements. */
 int arkv_fp8_encode(const float *x, uint8_t *out, size_t n, arkv_stream_t stream);
 
+/* Allocation-free tier reassignment.  The paper has no counterpart: this is an
+ * interface for callers that cannot allocate device memory when they reassign --
+ * code running while a CUDA graph is captured (cudaMalloc is not a stream
+ * operation a capture can record), serving engines that reserve all device
+ * memory at start-up and forbid later allocations, plugins whose host framework
+ * owns the allocator.  It computes exactly what arkv_reassign computes, with the
+ * same arguments except the workspace: its scratch is a static device array of
+ * ARKV_NOALLOC_SCRATCH_BYTES that every GPU loading this library holds until the
+ * process exits.  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture.  All calls share the array and it keeps the last call's
+ * contents (nothing in it needs to start at zero); calls whose executions overlap
+ * on the GPU race on it, so the caller must order them.  A layer whose scratch
+ * (arkv_workspace_bytes(cfg, ARKV_WS_REASSIGN, 0)) exceeds the array is rejected
+ * with ARKV_EINVAL and a message; it calls no allocating routine. */
+#define ARKV_NOALLOC_SCRATCH_BYTES (24u << 20)
+int arkv_reassign_noalloc(const arkv_cfg *cfg, int32_t step, float r, const int32_t *ctx_len,
+                          arkv_layer_cache *cache, uint8_t *tier_dbg, arkv_stream_t stream);
+
 /* Message of the calling thread's last failure ("" if none). */
 const char *arkv_last_error_string(void);
 

@@ -16,6 +16,7 @@ ARKV_OK, ARKV_EINVAL, ARKV_ECAPACITY, ARKV_ECUDA = 0, -1, -2, -3
 ARKV_STATUS_BF16_FULL, ARKV_STATUS_FP8_FULL = 1, 2
 ARKV_TIER_ORIGINAL, ARKV_TIER_QUANTIZED, ARKV_TIER_EVICTED = 0, 1, 2
 ARKV_WS_DECODE, ARKV_WS_REASSIGN, ARKV_WS_PREFILL = 0, 1, 2
+ARKV_NOALLOC_SCRATCH_BYTES = 24 << 20
 
 
 class arkv_cfg(ctypes.Structure):
@@ -52,6 +53,7 @@ _SIG = {
     "arkv_reassign": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_float, _P, _P, _P, _P,
                                      ctypes.c_size_t, _P]),
     "arkv_fp8_encode": (ctypes.c_int, [_P, _P, ctypes.c_size_t, _P]),
+    "arkv_reassign_noalloc": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_float, _P, _P, _P, _P]),
     "arkv_last_error_string": (ctypes.c_char_p, []),
 }
 
@@ -132,6 +134,12 @@ def arkv_score_update(cfg, step, ctx_len, cache, ws, ws_bytes, stream, check=Tru
 def arkv_reassign(cfg, step, r, ctx_len, cache, tier_dbg, ws, ws_bytes, stream, check=True) -> int:
     rc = lib().arkv_reassign(_ref(cfg), step, r, ctx_len, _ref(cache), tier_dbg, ws, ws_bytes, stream)
     return _check("arkv_reassign", rc) if check else rc
+
+
+def arkv_reassign_noalloc(cfg, step, r, ctx_len, cache, tier_dbg, stream, check=True) -> int:
+    """arkv_reassign without a workspace (scratch in the library's static device array)."""
+    rc = lib().arkv_reassign_noalloc(_ref(cfg), step, r, ctx_len, _ref(cache), tier_dbg, stream)
+    return _check("arkv_reassign_noalloc", rc) if check else rc
 
 
 def arkv_fp8_encode(x, out, n, stream, check=True) -> int:

@@ -94,6 +94,8 @@ PrefillWs prefill_ws(const arkv::LayerDims& d, int n_stride) {
 
 }  // namespace
 
+void arkv::set_last_error(const char* msg) { snprintf(g_err, sizeof g_err, "%s", msg); }
+
 extern "C" {
 
 const char* arkv_last_error_string(void) { return g_err; }

@@ -205,6 +205,9 @@ cudaError_t launch_prefill_stats(const PrefillParams& p, cudaStream_t s);
 
 cudaError_t launch_fp8_encode(const float* x, uint8_t* out, size_t n, cudaStream_t s);
 
+// Replace the calling thread's last-error message (see arkv_last_error_string).
+void set_last_error(const char* msg);
+
 // Raise a kernel's dynamic shared-memory limit to the device's opt-in maximum,
 // once per (kernel, device); later launches (including ones being captured into a
 // CUDA graph) then only launch.
