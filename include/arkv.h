@@ -63,6 +63,7 @@ typedef struct CUstream_st *arkv_stream_t;   /* same type as cudaStream_t */
 
 #define ARKV_STATUS_BF16_FULL  1   /* an append found the bf16 segment full; token dropped */
 #define ARKV_STATUS_FP8_FULL   2   /* a reassignment found the fp8 segment full; demotion became eviction */
+#define ARKV_STATUS_TIMEOUT    4   /* a kernel gave up waiting for its own bulk copy (a bug, never expected) */
 
 #define ARKV_TIER_ORIGINAL   0
 #define ARKV_TIER_QUANTIZED  1

@@ -36,7 +36,8 @@ def _stale() -> bool:
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not _stale():
         return LIB
-    cmd = [NVCC, *FLAGS, *(["-Xptxas", "-v"] if verbose else []), *sources(), "-o", LIB + ".tmp"]
+    extra = os.environ.get("ARKV_NVCC_EXTRA", "").split()   # e.g. -DARKV_STAGES=2
+    cmd = [NVCC, *FLAGS, *extra, *(["-Xptxas", "-v"] if verbose else []), *sources(), "-o", LIB + ".tmp"]
     subprocess.run(cmd, check=True)
     os.replace(LIB + ".tmp", LIB)
     return LIB

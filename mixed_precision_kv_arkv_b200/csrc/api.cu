@@ -213,7 +213,7 @@ int arkv_decode_attn(const arkv_cfg* cfg, int32_t step, const uint16_t* q, const
     p.nsplit_o = w.nsplit_o;
     p.nsplit_q = w.nsplit_q;
     p.inv_sqrt_d = 1.0 / sqrt((double)d.D);
-    const cudaError_t e = arkv::launch_decode_attn(p, (cudaStream_t)stream);
+    const cudaError_t e = arkv::launch_decode_attn(p, (cudaStream_t)stream);   // also encodes the tensor maps
     return e == cudaSuccess ? ARKV_OK : cuda_fail(e, "arkv_decode_attn");
 }
 

@@ -1,6 +1,7 @@
 // Internal declarations shared by the libarkv translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
@@ -117,6 +118,8 @@ struct LayerDims {
 };
 
 struct AttnParams {
+    CUtensorMap tm_k16, tm_v16;   // [R*cap_bf16][D] bf16, boxes of 16 rows x 128 bytes, 128B swizzle
+    CUtensorMap tm_k8, tm_v8;     // [R*cap_fp8][D] E4M3, boxes of 16 rows x min(D,128) bytes
     LayerDims d;
     int step;
     const uint16_t* q;
@@ -154,7 +157,7 @@ struct DecodeWs {
 };
 DecodeWs decode_ws_layout(const LayerDims& d);
 
-cudaError_t launch_decode_attn(const AttnParams& p, cudaStream_t s);
+cudaError_t launch_decode_attn(AttnParams& p, cudaStream_t s);   // fills the tensor maps
 cudaError_t launch_score_update(const ScoreParams& p, cudaStream_t s);
 
 struct ReassignParams {
@@ -226,6 +229,9 @@ cudaError_t allow_max_dyn_smem(K kernel, unsigned char (&done)[64]) {
     // static and dynamic shared memory share the per-block limit
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              optin - (int)fa.sharedSizeBytes);
+    if (e == cudaSuccess)   // ask for the largest shared-memory carveout, so that occupancy is not cut by L1
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
     if (e == cudaSuccess && dev < 64) __atomic_store_n(&done[dev], 1, __ATOMIC_RELEASE);
     return e;
 }
