@@ -16,7 +16,6 @@ constexpr int kAttnThreads = 128;      // decode attention CTA: 4 warps
 constexpr int kSplitBf16 = 256;        // bf16 tokens per decode CTA
 constexpr int kSplitFp8 = 512;         // fp8 tokens per decode CTA
 constexpr int kRowThreads = 1024;      // one CTA per row for selection / compaction
-constexpr int kScoreSlotsPerCta = 1024;
 
 // ------------------------------------------------------------------ numerics
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

@@ -618,37 +618,38 @@ __global__ void __launch_bounds__(4 * D) merge_kernel(const AttnParams p) {
     }
 }
 
-__global__ void score_update_kernel(const ScoreParams p) {
+// One thread per live slot: x = sum over the group's heads of exp((raw - M)/sqrt(D)) / L,
+// then one Welford step with the token's observation count.
+__global__ void __launch_bounds__(256) score_update_kernel(const ScoreParams p) {
     const LayerDims& d = p.d;
     const int row = blockIdx.y, b = row / d.hkv;
     __shared__ float2 sml[4];   // final (max, sum) of every head
-    if (threadIdx.x < 4) sml[threadIdx.x] = p.ml[(size_t)row * 4 + threadIdx.x];
+    if (threadIdx.x < 4) sml[threadIdx.x] = __ldg(&p.ml[(size_t)row * 4 + threadIdx.x]);
     __syncthreads();
-    const int n16 = min(max(p.c.n_bf16[row], 0), d.cap_o);
-    const int n8 = min(max(p.c.n_fp8[row], 0), d.cap_q);
-    const int n0 = p.ctx_len[b];
-    const int i0 = blockIdx.x * kScoreSlotsPerCta;
-    const int i1 = min(i0 + kScoreSlotsPerCta, n16 + n8);
-    for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
-        const bool bf = i < n16;
-        const size_t sl = bf ? (size_t)row * d.cap_o + i : (size_t)row * d.cap_q + (i - n16);
-        const float4 lg = bf ? reinterpret_cast<const float4*>(p.logit16)[sl]
-                             : reinterpret_cast<const float4*>(p.logit8)[sl];
-        const float lv[4] = {lg.x, lg.y, lg.z, lg.w};
-        double x = 0.0;
-        for (int h = 0; h < d.G; ++h)
-            x += (double)exp_scaled(lv[h], sml[h].x, p.inv_sqrt_d) / (double)sml[h].y;
-        const int pos = bf ? p.c.pos16[sl] : p.c.pos8[sl];
-        const int n = obs_count_after(pos, n0, p.step, d.n_obs);
-        float* mu = bf ? p.c.mu16 + sl : p.c.mu8 + sl;
-        float* m2 = bf ? p.c.m2_16 + sl : p.c.m2_8 + sl;
-        double mv = *mu, qv = *m2;
-        const double dl = x - mv;
-        mv += dl / (double)n;
-        qv += dl * (x - mv);
-        *mu = (float)mv;
-        *m2 = (float)qv;
-    }
+    const int n16 = min(max(__ldg(&p.c.n_bf16[row]), 0), d.cap_o);
+    const int n8 = min(max(__ldg(&p.c.n_fp8[row]), 0), d.cap_q);
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n16 + n8) return;
+    const bool bf = i < n16;
+    const size_t sl = bf ? (size_t)row * d.cap_o + i : (size_t)row * d.cap_q + (i - n16);
+    const float4 lg = __ldg(bf ? reinterpret_cast<const float4*>(p.logit16) + sl
+                               : reinterpret_cast<const float4*>(p.logit8) + sl);
+    const int pos = __ldg(bf ? p.c.pos16 + sl : p.c.pos8 + sl);
+    float* __restrict__ mu = bf ? p.c.mu16 + sl : p.c.mu8 + sl;
+    float* __restrict__ m2 = bf ? p.c.m2_16 + sl : p.c.m2_8 + sl;
+    const float mu_old = *mu, m2_old = *m2;
+    const float lv[4] = {lg.x, lg.y, lg.z, lg.w};
+    double x = 0.0;
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+        if (h < d.G) x += (double)exp_scaled(lv[h], sml[h].x, p.inv_sqrt_d) / (double)sml[h].y;
+    const int n = obs_count_after(pos, __ldg(&p.ctx_len[b]), p.step, d.n_obs);
+    double mv = mu_old, qv = m2_old;
+    const double dl = x - mv;
+    mv += dl / (double)n;
+    qv += dl * (x - mv);
+    *mu = (float)mv;
+    *m2 = (float)qv;
 }
 
 // ------------------------------------------------------------------ tensor maps
@@ -731,7 +732,7 @@ cudaError_t launch_decode_attn(AttnParams& p, cudaStream_t s) {
 }
 
 cudaError_t launch_score_update(const ScoreParams& p, cudaStream_t s) {
-    const dim3 grid((p.d.cap_o + p.d.cap_q + kScoreSlotsPerCta - 1) / kScoreSlotsPerCta, p.d.R);
+    const dim3 grid((p.d.cap_o + p.d.cap_q + 255) / 256, p.d.R);
     score_update_kernel<<<grid, 256, 0, s>>>(p);
     return cudaGetLastError();
 }
