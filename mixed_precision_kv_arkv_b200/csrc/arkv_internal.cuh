@@ -119,7 +119,6 @@ struct LayerDims {
 struct AttnParams {
     CUtensorMap tm_k16, tm_v16;   // [R*cap_bf16][D] bf16, boxes of 16 rows x 128 bytes, 128B swizzle
     CUtensorMap tm_k8, tm_v8;     // [R*cap_fp8][D] E4M3, boxes of 16 rows x min(D,128) bytes
-    CUtensorMap tm_q;             // [B*Hq][D] bf16 query rows (head_dim 128 path), boxes of 4 rows
     LayerDims d;
     int step;
     const uint16_t* q;
@@ -130,8 +129,8 @@ struct AttnParams {
     float* o;
     float* logit16;     // [R][cap_o][4]
     float* logit8;      // [R][cap_q][4]
-    float* part_o;      // [R][nsplit][2 slots][4][D]
-    float2* part_ml;    // [R][nsplit][2 slots][4]
+    float* part_o;      // [R][nsplit][4][D]
+    float2* part_ml;    // [R][nsplit][4]
     float2* ml;         // [R][4]  final (max, sum) per head
     unsigned* counter;  // [R]
     int nsplit_o, nsplit_q;
@@ -158,7 +157,6 @@ struct DecodeWs {
 DecodeWs decode_ws_layout(const LayerDims& d);
 
 cudaError_t launch_decode_attn(AttnParams& p, cudaStream_t s);   // fills the tensor maps
-cudaError_t launch_decode_attn_tc_kernel(const AttnParams& p, int ctas, cudaStream_t s);   // head_dim 128
 cudaError_t launch_score_update(const ScoreParams& p, cudaStream_t s);
 
 struct ReassignParams {

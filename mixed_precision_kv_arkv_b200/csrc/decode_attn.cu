@@ -526,7 +526,7 @@ __global__ void __launch_bounds__(32 * kWarps) decode_attn_kernel(const __grid_c
         if (w == 0) sm_max[h] = M;
     }
     __syncthreads();
-    const size_t pb = ((size_t)row * nsplit + split) * 2;   // partial slot 0; slot 1 stays empty
+    const size_t pb = (size_t)row * nsplit + split;
     for (int idx = tid; idx < 4 * D; idx += blockDim.x) {
         const int h = idx / D, dd = idx - h * D;
         float O = 0.f;
@@ -538,16 +538,14 @@ __global__ void __launch_bounds__(32 * kWarps) decode_attn_kernel(const __grid_c
 #pragma unroll
             for (int w = 0; w < kWarps; ++w) L = fmaf(sm_l[w][h], sm_w[w][h], L);
             p.part_ml[pb * 4 + h] = make_float2(sm_max[h], L);
-            p.part_ml[(pb + 1) * 4 + h] = make_float2(kNegInf, 0.f);
         }
     }
 }
 
-// Merges the partials of one (row, head): every live split has two partial slots
-// (the second holds the rest of a split cut between two CTAs, or is empty: sum 0).
-// M = max of the partial maxima, L = sum of l_s exp((m_s - M)/sqrt(D)),
-// o = sum of o_s exp(..) / L.  4 x D threads: thread (q, d) sums the partials
-// s = q mod 4 of output dim d, so every thread has only a few loads in flight.  Also publishes (M, L) for
+// Merges the split partials of one (row, head): M = max of the split maxima,
+// L = sum of l_s exp((m_s - M)/sqrt(D)), o = sum of o_s exp(..) / L.  4 x D
+// threads: thread (q, d) sums the splits s = q mod 4 of output dim d, so every
+// thread has only a few independent loads in flight.  Also publishes (M, L) for
 // the score update and advances the row's bf16 count past the appended token.
 template <int D>
 __global__ void __launch_bounds__(4 * D) merge_kernel(const AttnParams p) {
@@ -556,7 +554,7 @@ __global__ void __launch_bounds__(4 * D) merge_kernel(const AttnParams p) {
     const int b = row / d.hkv, g = row - b * d.hkv;
     const int nsplit = p.nsplit_o + p.nsplit_q;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    extern __shared__ float sm_w[];                  // [2 nlive] weights, then [4][D] partial sums
+    extern __shared__ float sm_w[];                  // [nlive] weights, then [4][D] partial sums
     __shared__ float sm_red[4 * D / 32];
     __shared__ float sm_ML[2];
     const double inv = p.inv_sqrt_d;
@@ -565,16 +563,11 @@ __global__ void __launch_bounds__(4 * D) merge_kernel(const AttnParams p) {
     const int nl16 = n16_old + (n16_old < d.cap_o ? 1 : 0);
     const int n8 = min(max(p.c.n_fp8[row], 0), d.cap_q);
     const int nlo = (nl16 + kSplitBf16 - 1) / kSplitBf16, nlive = nlo + (n8 + kSplitFp8 - 1) / kSplitFp8;
-    // partial k of the row: slot k & 1 of live split k >> 1
-    auto rec = [&](int k) { const int j = k >> 1; return (j < nlo ? j : p.nsplit_o + (j - nlo)) * 2 + (k & 1); };
-    const int nrec = 2 * nlive;
-    const float2* pml = p.part_ml + (size_t)row * nsplit * 2 * 4;
+    auto split_of = [&](int j) { return j < nlo ? j : p.nsplit_o + (j - nlo); };
+    const float2* pml = p.part_ml + (size_t)row * nsplit * 4;
 
     float mloc = kNegInf;
-    for (int s = tid; s < nrec; s += blockDim.x) {
-        const float2 ml = pml[rec(s) * 4 + h];
-        if (ml.y > 0.f) mloc = fmaxf(mloc, ml.x);
-    }
+    for (int s = tid; s < nlive; s += blockDim.x) mloc = fmaxf(mloc, pml[split_of(s) * 4 + h].x);
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(kFull, mloc, m));
     if (lane == 0) sm_red[warp] = mloc;
@@ -587,8 +580,8 @@ __global__ void __launch_bounds__(4 * D) merge_kernel(const AttnParams p) {
     __syncthreads();
     const float M = sm_ML[0];
     float lloc = 0.f;
-    for (int s = tid; s < nrec; s += blockDim.x) {
-        const float2 ml = pml[rec(s) * 4 + h];
+    for (int s = tid; s < nlive; s += blockDim.x) {
+        const float2 ml = pml[split_of(s) * 4 + h];
         const float wt = (ml.y > 0.f && M != kNegInf) ? exp_scaled(ml.x, M, inv) : 0.f;
         sm_w[s] = wt;
         lloc = fmaf(ml.y, wt, lloc);
@@ -605,14 +598,14 @@ __global__ void __launch_bounds__(4 * D) merge_kernel(const AttnParams p) {
         p.ml[(size_t)row * 4 + h] = make_float2(M, L);
     }
     const int q = tid / D, dd = tid - q * D;
-    const float* po = p.part_o + (size_t)row * nsplit * 2 * 4 * D + (size_t)h * D + dd;
+    const float* po = p.part_o + (size_t)row * nsplit * 4 * D + (size_t)h * D + dd;
     float acc = 0.f;
 #pragma unroll 4
-    for (int s = q; s < nrec; s += 4) {
+    for (int s = q; s < nlive; s += 4) {
         const float wt = sm_w[s];
-        if (wt != 0.f) acc = fmaf(po[(size_t)rec(s) * 4 * D], wt, acc);
+        if (wt != 0.f) acc = fmaf(po[(size_t)split_of(s) * 4 * D], wt, acc);
     }
-    float* sm_acc = sm_w + 2 * nsplit;
+    float* sm_acc = sm_w + nsplit;
     sm_acc[q * D + dd] = acc;
     __syncthreads();
     if (q == 0 && h < d.G) {
@@ -676,12 +669,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 2-D map over rows x D elements of one cache array, 16-row boxes of `box_inner`
 // elements.
 bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, int D, long long rows,
-              int box_inner, CUtensorMapSwizzle sw, int box_rows = 16) {
+              int box_inner, CUtensorMapSwizzle sw) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)D * elem_bytes};
-    cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows};
+    cuuint32_t box[2] = {(cuuint32_t)box_inner, 16};
     cuuint32_t es[2] = {1, 1};
     return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -698,8 +691,8 @@ DecodeWs decode_ws_layout(const LayerDims& d) {
     size_t off = 0;
     w.counter = off; off = al(off + sizeof(unsigned) * d.R);
     w.ml = off;      off = al(off + sizeof(float2) * d.R * 4);
-    w.part_ml = off; off = al(off + sizeof(float2) * d.R * ns * 2 * 4);
-    w.part_o = off;  off = al(off + sizeof(float) * d.R * ns * 2 * 4 * d.D);
+    w.part_ml = off; off = al(off + sizeof(float2) * d.R * ns * 4);
+    w.part_o = off;  off = al(off + sizeof(float) * d.R * ns * 4 * d.D);
     w.logit16 = off; off = al(off + sizeof(float) * 4 * (size_t)d.R * d.cap_o);
     w.logit8 = off;  off = al(off + sizeof(float) * 4 * (size_t)d.R * d.cap_q);
     w.total = off;
@@ -709,49 +702,32 @@ DecodeWs decode_ws_layout(const LayerDims& d) {
 cudaError_t launch_decode_attn(AttnParams& p, cudaStream_t s) {
     const LayerDims& d = p.d;
     const int D = d.D;
-    const int nsplit = p.nsplit_o + p.nsplit_q;
-    const dim3 mgrid(d.R, d.G);
-    const size_t mdyn = sizeof(float) * (2 * (size_t)nsplit + 4 * (size_t)D);
-    if (mdyn > 48 * 1024) return cudaErrorInvalidValue;
-    if (D == 128) {
-        // tensor-core path: 128-row boxes, one persistent CTA per SM
-        const long long R16 = (long long)d.R * d.cap_o, R8 = (long long)d.R * d.cap_q;
-        const bool ok =
-            make_map(&p.tm_k16, p.c.k16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, R16, 64, CU_TENSOR_MAP_SWIZZLE_128B, 128) &&
-            make_map(&p.tm_v16, p.c.v16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, R16, 64, CU_TENSOR_MAP_SWIZZLE_128B, 128) &&
-            make_map(&p.tm_k8, p.c.k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D, R8, 128, CU_TENSOR_MAP_SWIZZLE_128B, 128) &&
-            make_map(&p.tm_v8, p.c.v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D, R8, 128, CU_TENSOR_MAP_SWIZZLE_128B, 128) &&
-            make_map(&p.tm_q, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, (long long)d.batch * d.hq, 64,
-                     CU_TENSOR_MAP_SWIZZLE_128B, 4);
-        if (!ok) return cudaErrorInvalidValue;
-        static int sms[64];
-        int dev = 0;
-        cudaError_t e = cudaGetDevice(&dev);
-        if (e != cudaSuccess) return e;
-        if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-        if (sms[dev] == 0 && (e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-            return e;
-        const long long units = (long long)nsplit * d.R;
-        const int ctas = (int)(units < sms[dev] ? units : sms[dev]);
-        if ((e = launch_decode_attn_tc_kernel(p, ctas, s)) != cudaSuccess) return e;
-        merge_kernel<128><<<mgrid, 4 * 128, mdyn, s>>>(p);
-        return cudaGetLastError();
-    }
     const bool ok = make_map(&p.tm_k16, p.c.k16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, (long long)d.R * d.cap_o, 64,
                              CU_TENSOR_MAP_SWIZZLE_128B) &&
                     make_map(&p.tm_v16, p.c.v16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, (long long)d.R * d.cap_o, 64,
                              CU_TENSOR_MAP_SWIZZLE_128B) &&
                     make_map(&p.tm_k8, p.c.k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D, (long long)d.R * d.cap_q, D,
-                             CU_TENSOR_MAP_SWIZZLE_64B) &&
+                             D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) &&
                     make_map(&p.tm_v8, p.c.v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D, (long long)d.R * d.cap_q, D,
-                             CU_TENSOR_MAP_SWIZZLE_64B);
+                             D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
     if (!ok) return cudaErrorInvalidValue;
-    static unsigned char done64[64];
+    const int nsplit = p.nsplit_o + p.nsplit_q;
+    const dim3 mgrid(d.R, d.G);
+    const size_t mdyn = sizeof(float) * ((size_t)nsplit + 4 * (size_t)D);
+    if (mdyn > 48 * 1024) return cudaErrorInvalidValue;
+    static unsigned char done128[64], done64[64];
     const dim3 grid(nsplit, d.R);
-    const cudaError_t e = allow_max_dyn_smem(decode_attn_kernel<64>, done64);
-    if (e != cudaSuccess) return e;
-    decode_attn_kernel<64><<<grid, 32 * kWarps, Smem<64>::kBytes, s>>>(p);
-    merge_kernel<64><<<mgrid, 4 * 64, mdyn, s>>>(p);
+    if (D == 128) {
+        const cudaError_t e = allow_max_dyn_smem(decode_attn_kernel<128>, done128);
+        if (e != cudaSuccess) return e;
+        decode_attn_kernel<128><<<grid, 32 * kWarps, Smem<128>::kBytes, s>>>(p);
+        merge_kernel<128><<<mgrid, 4 * 128, mdyn, s>>>(p);
+    } else {
+        const cudaError_t e = allow_max_dyn_smem(decode_attn_kernel<64>, done64);
+        if (e != cudaSuccess) return e;
+        decode_attn_kernel<64><<<grid, 32 * kWarps, Smem<64>::kBytes, s>>>(p);
+        merge_kernel<64><<<mgrid, 4 * 64, mdyn, s>>>(p);
+    }
     return cudaGetLastError();
 }
 
