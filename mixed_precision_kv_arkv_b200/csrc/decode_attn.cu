@@ -22,8 +22,10 @@
 // carry tokens 4t, 4t+1 | 4t+2, 4t+3 and P's rows are permuted to match).  The
 // per-token K scale multiplies the finished logit; the V scale is folded into P
 // relative to the largest V scale the warp will meet, and the constant comes
-// back out of the warp's partial.  The softmax runs in float32 registers; raw
-// logits go to the workspace for the score update.  The CTA combines its warps
+// back out of the warp's partial.  The softmax runs in float32 registers with a
+// reference maximum that moves only when a logit exceeds it by 2^8 (so most
+// tiles need no cross-lane reduction); raw logits go to the workspace for the
+// score update.  The CTA combines its warps
 // into one (max, sum, unnormalised o) partial per split; merge_kernel combines a
 // row's splits and writes o.
 #include <math.h>
@@ -169,7 +171,7 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair) {
 // Fragment conventions of m16n8k16: g = lane / 4, t = lane % 4.  ks: the stage
 // (K tile, V tile at +VOFF); tokens t0 .. t0+15 of a segment ending at seg_end.
 // sk*/sv*: the FP8 scales of this lane's tokens t0+g, t0+g+8 (1 for bf16);
-// vnorm: the warp's V-scale normaliser (FP8).
+// vnorm: the warp's V-scale normaliser (FP8): 64 / the largest V scale of the warp's tiles.
 template <int D, bool FP8>
 __device__ __forceinline__ void attend_tile(const char* ks, int t0, int seg_end, int G, float c2, float skA,
                                             float skB, float svA, float svB, float vnorm, float* logit_row,
@@ -223,35 +225,42 @@ __device__ __forceinline__ void attend_tile(const char* ks, int t0, int seg_end,
         if (okB) *reinterpret_cast<float2*>(logit_row + (size_t)tokB * 4 + 2 * t) = make_float2(s[2], s[3]);
     }
     const bool v0 = okA && h0ok, v1 = okA && h1ok, v2 = okB && h0ok, v3 = okB && h1ok;
-    float mx0 = fmaxf(v0 ? s[0] : kNegInf, v2 ? s[2] : kNegInf);
-    float mx1 = fmaxf(v1 ? s[1] : kNegInf, v3 ? s[3] : kNegInf);
+    // online softmax for heads 2t, 2t+1 (uniform over the lanes sharing t), with a
+    // lazy reference: it moves only when a logit exceeds it by more than 8 in log2
+    // units, so probabilities stay below 2^8 and most tiles skip the reductions
+    const bool need = (v0 && (s[0] - m_run[0]) * c2 > 8.f) || (v1 && (s[1] - m_run[1]) * c2 > 8.f) ||
+                      (v2 && (s[2] - m_run[0]) * c2 > 8.f) || (v3 && (s[3] - m_run[1]) * c2 > 8.f);
+    float al0 = 1.f, al1 = 1.f;
+    if (__any_sync(kFull, need)) {
+        float mx0 = fmaxf(v0 ? s[0] : kNegInf, v2 ? s[2] : kNegInf);
+        float mx1 = fmaxf(v1 ? s[1] : kNegInf, v3 ? s[3] : kNegInf);
 #pragma unroll
-    for (int m = 4; m < 32; m <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, m));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, m));
-    }
-    // online softmax for heads 2t, 2t+1 (uniform over the lanes sharing t)
-    const float n0 = fmaxf(m_run[0], mx0), n1 = fmaxf(m_run[1], mx1);
-    const float al0 = (n0 == kNegInf || m_run[0] == n0) ? 1.f : exp2f((m_run[0] - n0) * c2);
-    const float al1 = (n1 == kNegInf || m_run[1] == n1) ? 1.f : exp2f((m_run[1] - n1) * c2);
-    m_run[0] = n0;
-    m_run[1] = n1;
-    const float p0 = v0 ? exp2f((s[0] - n0) * c2) : 0.f;
-    const float p1 = v1 ? exp2f((s[1] - n1) * c2) : 0.f;
-    const float p2 = v2 ? exp2f((s[2] - n0) * c2) : 0.f;
-    const float p3 = v3 ? exp2f((s[3] - n1) * c2) : 0.f;
-    l_run[0] = fmaf(l_run[0], al0, p0 + p2);
-    l_run[1] = fmaf(l_run[1], al1, p1 + p3);
-    // o columns of this lane: heads 2 (t & 1), +1, high (t < 2) or low (t >= 2) half
-    const float b0 = __shfl_xor_sync(kFull, al0, 2), b1 = __shfl_xor_sync(kFull, al1, 2);
-    const float oa0 = t < 2 ? al0 : b0, oa1 = t < 2 ? al1 : b1;
-    if (__any_sync(kFull, oa0 != 1.f || oa1 != 1.f)) {   // a running max moved: rescale o
+        for (int m = 4; m < 32; m <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, m));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, m));
+        }
+        const float n0 = fmaxf(m_run[0], mx0), n1 = fmaxf(m_run[1], mx1);
+        al0 = (n0 == kNegInf || m_run[0] == n0) ? 1.f : exp2f((m_run[0] - n0) * c2);
+        al1 = (n1 == kNegInf || m_run[1] == n1) ? 1.f : exp2f((m_run[1] - n1) * c2);
+        m_run[0] = n0;
+        m_run[1] = n1;
+        // o columns of this lane: heads 2 (t & 1), +1, high (t < 2) or low (t >= 2) half
+        const float b0 = __shfl_xor_sync(kFull, al0, 2), b1 = __shfl_xor_sync(kFull, al1, 2);
+        const float oa0 = t < 2 ? al0 : b0, oa1 = t < 2 ? al1 : b1;
+        if (__any_sync(kFull, oa0 != 1.f || oa1 != 1.f)) {   // a reference moved: rescale o
 #pragma unroll
-        for (int mt = 0; mt < KB; ++mt) {
-            oacc[mt][0] *= oa0; oacc[mt][1] *= oa1;
-            oacc[mt][2] *= oa0; oacc[mt][3] *= oa1;
+            for (int mt = 0; mt < KB; ++mt) {
+                oacc[mt][0] *= oa0; oacc[mt][1] *= oa1;
+                oacc[mt][2] *= oa0; oacc[mt][3] *= oa1;
+            }
         }
     }
+    const float p0 = v0 ? exp2f((s[0] - m_run[0]) * c2) : 0.f;
+    const float p1 = v1 ? exp2f((s[1] - m_run[1]) * c2) : 0.f;
+    const float p2 = v2 ? exp2f((s[2] - m_run[0]) * c2) : 0.f;
+    const float p3 = v3 ? exp2f((s[3] - m_run[1]) * c2) : 0.f;
+    l_run[0] = fmaf(l_run[0], al0, p0 + p2);
+    l_run[1] = fmaf(l_run[1], al1, p1 + p3);
     // P (times V scale / normaliser for FP8) to shared memory, [token][head]
     float w0 = p0, w1 = p1, w2 = p2, w3 = p3;
     if constexpr (FP8) {
@@ -293,8 +302,9 @@ __device__ __forceinline__ void attend_tile(const char* ks, int t0, int seg_end,
     // past the segment end the tile holds stale slots or zero fill: P is 0 there,
     // and a partial tile also zeroes those V elements so that no stale bit pattern
     // can reach the accumulator (same token order as the B fragment)
+    const bool partial = t0 + 16 > seg_end;   // warp-uniform
     uint32_t m01 = 0xffffffffu, m23 = 0xffffffffu;
-    if (t0 + 16 > seg_end) {
+    if (partial) {
         m01 = (t0 + ta < seg_end ? 0xffffu : 0u) | (t0 + ta + 1 < seg_end ? 0xffff0000u : 0u);
         m23 = (t0 + tb < seg_end ? 0xffffu : 0u) | (t0 + tb + 1 < seg_end ? 0xffff0000u : 0u);
     }
@@ -315,7 +325,9 @@ __device__ __forceinline__ void attend_tile(const char* ks, int t0, int seg_end,
             const int byte = 2 * (16 * mt + 8 * ((lane >> 3) & 1));
             ldsm_x4_trans(a, vs + (byte >> 7) * 2048 + swz<128>(tok, byte & 127));
         }
-        a[0] &= m01; a[1] &= m01; a[2] &= m23; a[3] &= m23;
+        if (partial) {
+            a[0] &= m01; a[1] &= m01; a[2] &= m23; a[3] &= m23;
+        }
         mma16816<FP8>(oacc[mt], a, bb0, bb1);
     }
 }
@@ -445,7 +457,7 @@ __global__ void __launch_bounds__(32 * kWarps) decode_attn_kernel(const __grid_c
         }
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(kFull, vmax, m));
-        vnorm = vmax > 0.f ? 16384.f / vmax : 0.f;
+        vnorm = vmax > 0.f ? 64.f / vmax : 0.f;   // p < 2^8: p sv vnorm < 2^14, inside f16
         const int a = min(first + fg, d.cap_q - 1), c = min(first + fg + 8, d.cap_q - 1);
         nskA = __ldg(skb + a); nskB = __ldg(skb + c);
         nsvA = __ldg(svb + a); nsvB = __ldg(svb + c);
@@ -496,7 +508,7 @@ __global__ void __launch_bounds__(32 * kWarps) decode_attn_kernel(const __grid_c
         l_run[0] += __shfl_xor_sync(kFull, l_run[0], m);
         l_run[1] += __shfl_xor_sync(kFull, l_run[1], m);
     }
-    const float un = fp8 ? vmax * (1.f / 16384.f) : 1.f;
+    const float un = fp8 ? vmax * (1.f / 64.f) : 1.f;
 #pragma unroll
     for (int mt = 0; mt < KB; ++mt)
 #pragma unroll
@@ -565,6 +577,18 @@ __global__ void __launch_bounds__(4 * D) merge_kernel(const AttnParams p) {
     const int nlo = (nl16 + kSplitBf16 - 1) / kSplitBf16, nlive = nlo + (n8 + kSplitFp8 - 1) / kSplitFp8;
     auto split_of = [&](int j) { return j < nlo ? j : p.nsplit_o + (j - nlo); };
     const float2* pml = p.part_ml + (size_t)row * nsplit * 4;
+    // the partial outputs this thread sums (splits q, q + 4, ...) do not depend on
+    // the weights: their loads are issued first, so their latency overlaps the
+    // reductions below
+    const int q = tid / D, dd = tid - q * D;
+    const float* po = p.part_o + (size_t)row * nsplit * 4 * D + (size_t)h * D + dd;
+    constexpr int kPre = 12;
+    float pre[kPre];
+#pragma unroll
+    for (int k = 0; k < kPre; ++k) {
+        const int sidx = q + 4 * k;
+        pre[k] = sidx < nlive ? po[(size_t)split_of(sidx) * 4 * D] : 0.f;
+    }
 
     float mloc = kNegInf;
     for (int s = tid; s < nlive; s += blockDim.x) mloc = fmaxf(mloc, pml[split_of(s) * 4 + h].x);
@@ -597,11 +621,15 @@ __global__ void __launch_bounds__(4 * D) merge_kernel(const AttnParams p) {
         sm_ML[1] = L;
         p.ml[(size_t)row * 4 + h] = make_float2(M, L);
     }
-    const int q = tid / D, dd = tid - q * D;
-    const float* po = p.part_o + (size_t)row * nsplit * 4 * D + (size_t)h * D + dd;
+    __syncthreads();   // the weights
     float acc = 0.f;
+#pragma unroll
+    for (int k = 0; k < kPre; ++k) {
+        const int sidx = q + 4 * k;
+        if (sidx < nlive && sm_w[sidx] != 0.f) acc = fmaf(pre[k], sm_w[sidx], acc);
+    }
 #pragma unroll 4
-    for (int s = q; s < nlive; s += 4) {
+    for (int s = q + 4 * kPre; s < nlive; s += 4) {
         const float wt = sm_w[s];
         if (wt != 0.f) acc = fmaf(po[(size_t)split_of(s) * 4 * D], wt, acc);
     }
