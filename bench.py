@@ -57,9 +57,16 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# kernels one decode step of one layer launches: decode_attn_kernel and merge_kernel
+# (arkv_decode_attn), score_update_kernel (arkv_score_update); arkv_reassign adds
+# reassign_kernel every reassignment interval
+KERNELS_PER_LAYER_STEP = 3
+
+
 def kernel_traffic(kernel_file: str):
-    """DRAM bytes per launch of the decode kernel from the committed ncu summary, if
-    it was taken on the current kernel source (else None)."""
+    """DRAM bytes (read + write) of one arkv_decode_attn call -- its attention and
+    merge kernels -- from the committed ncu summary, if it was taken on the current
+    kernel source (else None)."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "decode_attn_traffic.txt")
     src = os.path.join(ROOT, "mixed_precision_kv_arkv_b200", "csrc", kernel_file)
@@ -283,7 +290,7 @@ def run_arkv(args, wl, rank, world, local_rank):
         if ev is not None:
             ev[1].record()
         abi.arkv_score_update(cfg, t, ctx.data_ptr(), c, x["ws_d"].ptr, x["ws_d"].nbytes, stream_ptr())
-        launches["n"] += 2
+        launches["n"] += KERNELS_PER_LAYER_STEP
         if (t + 1) % wl.reassign_interval == 0:
             abi.arkv_reassign(cfg, t, x["r"], ctx.data_ptr(), c, None, x["ws_r"].ptr, x["ws_r"].nbytes,
                               stream_ptr())
@@ -312,7 +319,7 @@ def run_arkv(args, wl, rank, world, local_rank):
     launches["n"] = 0
     for tt in range(t_value, t_value + K):
         for l in range(L):
-            launches["n"] += 2 + (1 if (tt + 1) % wl.reassign_interval == 0 else 0)
+            launches["n"] += KERNELS_PER_LAYER_STEP + (1 if (tt + 1) % wl.reassign_interval == 0 else 0)
     gpu_launches = launches["n"]
 
     # ---------- pass 2: end to end through host buffers
@@ -394,7 +401,8 @@ def run_arkv(args, wl, rank, world, local_rank):
         "hbm_gbs_step": step_bytes / (ms_value / K * 1e-3) / 1e9,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": kernel_traffic("decode_attn.cu"),
-                     "kernel": "decode_attn_kernel<128>" if D == 128 else "decode_attn_kernel<64>",
+                     "kernel": (f"arkv_decode_attn call: decode_attn_kernel<{D}> + merge_kernel<{D}> "
+                                "(timed together; algorithmic bytes are the attention's)"),
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                      else "fallback 6650 GB/s",
                      "bytes_per_launch": float(alg_bytes.mean()),
