@@ -57,6 +57,24 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def max_over_ranks(x: float, device, world: int) -> float:
+    """The largest of every rank's x (the job's time is its slowest rank's); x itself
+    when there is one rank."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(batch: int, steps: int, world: int, ms: float) -> float:
+    """Whole-job decode throughput: every rank decodes `batch` sequences per step
+    (independent replicas), timed by the slowest rank."""
+    return batch * steps * world / (ms * 1e-3)
+
+
 # kernels one decode step of one layer launches: decode_attn_kernel and merge_kernel
 # (arkv_decode_attn), score_update_kernel (arkv_score_update); arkv_reassign adds
 # reassign_kernel every reassignment interval
@@ -369,12 +387,7 @@ def run_arkv(args, wl, rank, world, local_rank):
             g.replay()
         b.record()
         torch.cuda.synchronize()
-        ms = a.elapsed_time(b)
-        if world > 1:
-            tm = torch.tensor([ms], device=dev)
-            dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-            ms = float(tm.item())
-        return ms
+        return max_over_ranks(a.elapsed_time(b), dev, world)
 
     with ClockSampler(local_rank) as clk:
         ms_value = timed(g_value)
@@ -392,8 +405,7 @@ def run_arkv(args, wl, rank, world, local_rank):
     step_bytes = float(alg_bytes.sum(-1).mean())
 
     status = sum(int(x["cache"].status.item()) for x in layers)
-    tokens = B * K * world
-    value = tokens / (ms_value * 1e-3)
+    value = job_tokens_per_s(B, K, world, ms_value)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": ms_value / K, "higher_is_better": True, "scaling": "weak",
@@ -413,7 +425,7 @@ def run_arkv(args, wl, rank, world, local_rank):
         "cache_status": status,
     }
     if not args.no_e2e:
-        line["e2e"] = {"value": tokens / (ms_e2e * 1e-3), "unit": "tokens/s",
+        line["e2e"] = {"value": job_tokens_per_s(B, K, world, ms_e2e), "unit": "tokens/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "ms_per_step": ms_e2e / K}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
