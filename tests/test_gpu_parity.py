@@ -181,7 +181,14 @@ SMALL_CLUSTER = workloads.QWEN3_8B.with_(name="small_clustered", cfg_id=13, laye
                                          hh_span_len=128)
 
 
-@pytest.mark.parametrize("wl", [SMALL_D128_G3, SMALL_RAGGED, SMALL_CLUSTER], ids=lambda w: w.name)
+# query groups of one and two heads (the unused columns of the query operand stay zero)
+SMALL_D128_G1 = workloads.LLAMA3_3B.with_(name="small_d128_g1", cfg_id=14, layers=1, batch=2, hq=4, hkv=4,
+                                          n_ctx=2500, n_ctx_min=2500, steps=8, reassign_interval=4)
+SMALL_D64_G2 = workloads.TINY.with_(name="small_d64_g2", cfg_id=15, hq=4, hkv=2, steps=8)
+
+
+@pytest.mark.parametrize("wl", [SMALL_D128_G3, SMALL_RAGGED, SMALL_CLUSTER, SMALL_D128_G1, SMALL_D64_G2],
+                         ids=lambda w: w.name)
 def test_small_workloads(cuda, wl):
     s = run_scenario(wl, wl.steps, cuda)
     print(wl.name, s)
