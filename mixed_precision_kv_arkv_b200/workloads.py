@@ -80,5 +80,15 @@ RAGGED = Workload("ragged_l32_b32_h32x8_d128_n4096to16384", 5, layers=32, batch=
                   reassign_interval=16, hh_frac=0.05)
 
 ALL = (TINY, LLAMA3_3B, LLAMA3_8B, QWEN3_8B, RAGGED)
-BY_NAME = {w.name: w for w in ALL}
+
+# The page's comparison axes on the LLaMA3-8B data (the same generator stream): the
+# uncompressed cache (every token bf16), eviction only (Base Origin, the ARKV budget
+# with no quantized tier) and quantization only (Base Quant: every non-window token
+# FP8, none evicted -- the budget covers them all).
+LLAMA3_8B_FULL = LLAMA3_8B.with_(name="llama3_8b_full_bf16", budget_frac=1.0, oq_ratio=1.0)
+LLAMA3_8B_BASE_ORIGIN = LLAMA3_8B.with_(name="llama3_8b_base_origin", oq_ratio=1.0)
+LLAMA3_8B_BASE_QUANT = LLAMA3_8B.with_(name="llama3_8b_base_quant", budget_frac=0.52, oq_ratio=0.0)
+MODES = (LLAMA3_8B_FULL, LLAMA3_8B_BASE_ORIGIN, LLAMA3_8B_BASE_QUANT)
+
+BY_NAME = {w.name: w for w in ALL + MODES}
 BY_ID = {w.cfg_id: w for w in ALL}
