@@ -367,8 +367,14 @@ __global__ void __launch_bounds__(32 * kWarps) decode_attn_kernel(const __grid_c
     constexpr int VOFF = SL::kTileBytes;
     constexpr int NB16 = D * 2 / 128;                // bf16 boxes per tile
     const LayerDims& d = p.d;
-    const int row = blockIdx.y, b = row / d.hkv, gk = row - b * d.hkv;
-    const int split = blockIdx.x, nsplit = p.nsplit_o + p.nsplit_q;
+    // CTA order, longest work first: the FP8 splits of every row (rows fastest), then
+    // the bf16 splits.  An FP8 split holds twice the tokens of a bf16 split and costs
+    // more per tile, so dispatching it last would leave the longest CTAs in the tail.
+    const int nq = p.nsplit_q * d.R, bid = blockIdx.x;
+    const int row = bid < nq ? bid % d.R : (bid - nq) % d.R;
+    const int split = bid < nq ? p.nsplit_o + bid / d.R : (bid - nq) / d.R;
+    const int b = row / d.hkv, gk = row - b * d.hkv;
+    const int nsplit = p.nsplit_o + p.nsplit_q;
     const bool fp8 = split >= p.nsplit_o;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int fg = lane >> 2, ft = lane & 3;
@@ -744,7 +750,8 @@ cudaError_t launch_decode_attn(AttnParams& p, cudaStream_t s) {
     const size_t mdyn = sizeof(float) * ((size_t)nsplit + 4 * (size_t)D);
     if (mdyn > 48 * 1024) return cudaErrorInvalidValue;
     static unsigned char done128[64], done64[64];
-    const dim3 grid(nsplit, d.R);
+    if ((long long)nsplit * d.R > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const dim3 grid(nsplit * d.R);   // one CTA per (split, row); order set in the kernel
     if (D == 128) {
         const cudaError_t e = allow_max_dyn_smem(decode_attn_kernel<128>, done128);
         if (e != cudaSuccess) return e;
