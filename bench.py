@@ -254,7 +254,7 @@ def run_arkv(args, wl, rank, world, local_rank):
     probe = make_cfg(B, Hq, Hkv, D, wl.window, wl.n_obs, wl.gamma, wl.budget_frac, 1, 1)
     ws_pre = Workspace(abi.arkv_workspace_bytes(probe, abi.ARKV_WS_PREFILL, wl.n_ctx), dev)
     stats = torch.zeros((L, 3), dtype=torch.float64, device=dev)
-    mu0 = torch.zeros((wl.rows, wl.n_ctx), dtype=torch.float32, device=dev)
+    mu0 = torch.zeros((wl.rows, wl.n_ctx), dtype=torch.float64, device=dev)
     m20 = torch.zeros_like(mu0)
     seed = rank
     for l in range(L):

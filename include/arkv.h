@@ -18,9 +18,9 @@
  * row = b * hkv + g, R = batch * hkv rows per layer.  Each row owns two segments
  * of slots, in no particular order:
  *   bf16 segment  k16, v16 [R][cap_bf16][D] bf16 bits, pos16 [R][cap_bf16] int32,
- *                 mu16, m2_16 [R][cap_bf16] float (Welford mean and M2);
+ *                 mu16, m2_16 [R][cap_bf16] double (Welford mean and M2);
  *   fp8 segment   k8, v8 [R][cap_fp8][D] E4M3 codes, sk, sv [R][cap_fp8] float
- *                 scales, pos8, mu8, m2_8 [R][cap_fp8];
+ *                 scales, pos8 int32, mu8, m2_8 double [R][cap_fp8];
  *   n_bf16 [R], n_fp8 [R]  live slots of each segment (slots 0 .. n-1).
  * The Welford count of a token is not stored: it is the number of observations
  * so far, a function of its position, its sequence's prefill length ctx_len[b],
@@ -89,11 +89,11 @@ typedef struct arkv_cfg {
 typedef struct arkv_layer_cache {
     uint16_t *k16, *v16;
     int32_t  *pos16;
-    float    *mu16, *m2_16;
+    double   *mu16, *m2_16;
     uint8_t  *k8, *v8;
     float    *sk, *sv;
     int32_t  *pos8;
-    float    *mu8, *m2_8;
+    double   *mu8, *m2_8;
     int32_t  *n_bf16, *n_fp8;
     int32_t  *status;       /* one int32, sticky ARKV_STATUS_* bits */
 } arkv_layer_cache;
@@ -124,14 +124,14 @@ int arkv_row_capacity(const arkv_cfg *cfg, int32_t n_ctx_max, float r,
  * (b, h, i); query_stats (device, nullable) receives them per query,
  * [batch][hq][n_obs][3] doubles.  Every key k < ctx_len[b] of row (b, g) gets the
  * Welford state of its observations x_k(i) = sum over the group's G heads of
- * p, i = 0..n_obs-1 with P_i >= k: mu0, m2_0 [R][n_ctx_max] floats.
+ * p, i = 0..n_obs-1 with P_i >= k: mu0, m2_0 [R][n_ctx_max] doubles.
  *   q_obs  [batch][hq][n_obs][D] bf16 bits (queries at the last n_obs positions)
  *   k      [batch][hkv][n_ctx_max][D] bf16 bits (keys 0 .. ctx_len[b]-1 used)
  *   ctx_len [batch] int32, n_obs <= ctx_len[b] <= n_ctx_max
  * Computed with float64 dot products and sums. */
 int arkv_prefill_stats(const arkv_cfg *cfg, const uint16_t *q_obs, const uint16_t *k,
                        int32_t n_ctx_max, const int32_t *ctx_len, double *stats_out,
-                       double *query_stats, float *mu0, float *m2_0, void *ws, size_t ws_bytes,
+                       double *query_stats, double *mu0, double *m2_0, void *ws, size_t ws_bytes,
                        arkv_stream_t stream);
 
 /* §2.가 / reading R-9: per-layer Original share from the layer statistics.
@@ -143,7 +143,8 @@ int arkv_oq_ratio(const double *stats, int32_t layers, double r_bar, float *r_ou
 
 /* §2.다: the reassignment right after prefill, and the initial pack.
  * Ranks the tokens of every row that are older than the window by
- * S = mu0 + gamma * m2_0 / n (n = min(n_obs, ctx_len[b] - pos)), keeps the budget's
+ * S = mu0 + gamma * m2_0 / n (n = min(n_obs, ctx_len[b] - pos), float64, ties by
+ * position), keeps the budget's
  * n_sel, makes the first n_o of them Original and quantizes the rest, evicts the
  * others, and writes the cache: bf16 segment = Originals + the W newest tokens,
  * fp8 segment = the Quantized tokens (codes = RNE_E4M3(x / s), s = amax / 448 in
@@ -154,8 +155,8 @@ int arkv_oq_ratio(const double *stats, int32_t layers, double r_bar, float *r_ou
  *   tier_out [R][n_ctx_max] uint8 ARKV_TIER_* per position (device, nullable).
  * Returns ARKV_ECAPACITY when cfg's capacities cannot hold the kept counts. */
 int arkv_quantize_pack(const arkv_cfg *cfg, float r, const uint16_t *k, const uint16_t *v,
-                       int32_t n_ctx_max, const int32_t *ctx_len, const float *mu0,
-                       const float *m2_0, arkv_layer_cache *cache, uint8_t *tier_out,
+                       int32_t n_ctx_max, const int32_t *ctx_len, const double *mu0,
+                       const double *m2_0, arkv_layer_cache *cache, uint8_t *tier_out,
                        void *ws, size_t ws_bytes, arkv_stream_t stream);
 
 /* §2.다 reconstruction: decode step `step` (0-based) of one layer.
@@ -178,20 +179,23 @@ int arkv_decode_attn(const arkv_cfg *cfg, int32_t step, const uint16_t *q, const
  * the token's observations: min(n_obs, ctx_len[b] - pos) + step for prefill
  * tokens, step - (pos - ctx_len[b]) for decode tokens, before this step.
  * S_k = mu_k + gamma * M2_k / n (population variance) is what arkv_reassign ranks.
- * Arithmetic in float64, state stored as float. */
+ * Arithmetic and state in float64. */
 int arkv_score_update(const arkv_cfg *cfg, int32_t step, const int32_t *ctx_len,
                       arkv_layer_cache *cache, const void *ws, size_t ws_bytes,
                       arkv_stream_t stream);
 
 /* §2.다: tier reassignment after decode step `step` (context N_t = ctx_len[b] +
  * step + 1).  The W newest positions stay Original.  The other live tokens are
- * ranked by (S descending, position ascending); the first n_sel (budget counts as
+ * ranked by (S descending, position ascending), S = mu + gamma * M2 / n evaluated in
+ * float64 and ranked on its 64-bit pattern; the first n_sel (budget counts as
  * in arkv_quantize_pack, with N_t) are kept; walking them in rank order, the first
  * n_o still in bf16 stay Original, the other kept bf16 tokens are quantized into
  * the fp8 segment, kept fp8 tokens keep their codes; all others are evicted.
  * Segments are compacted in place by moving tokens into vacated slots.
  *   tier_dbg [R][cap_bf16 + cap_fp8] uint8 (device, nullable): the new tier of
- *   every slot as it was before the call (bf16 slots first, then fp8 slots). */
+ *   every slot as it was before the call (bf16 slots first, then fp8 slots).  When
+ *   the fp8 segment cannot take every demotion (ARKV_STATUS_FP8_FULL), the
+ *   demotions that did not fit are evicted and reported as ARKV_TIER_EVICTED. */
 int arkv_reassign(const arkv_cfg *cfg, int32_t step, float r, const int32_t *ctx_len,
                   arkv_layer_cache *cache, uint8_t *tier_dbg, void *ws, size_t ws_bytes,
                   arkv_stream_t stream);
@@ -210,7 +214,10 @@ int arkv_fp8_encode(const float *x, uint8_t *out, size_t n, arkv_stream_t stream
  * ARKV_NOALLOC_SCRATCH_BYTES that every GPU loading this library holds until the
  * process exits.  The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call before
- * any stream capture.  All calls share the array and it keeps the last call's
+ * any stream capture.  The address is remembered together with the CUDA context
+ * it belongs to: after the context is destroyed and recreated (cudaDeviceReset),
+ * the next call looks it up again, so make that call outside a capture too.  All
+ * calls share the array and it keeps the last call's
  * contents (nothing in it needs to start at zero); calls whose executions overlap
  * on the GPU race on it, so the caller must order them.  A layer whose scratch
  * (arkv_workspace_bytes(cfg, ARKV_WS_REASSIGN, 0)) exceeds the array is rejected

@@ -22,20 +22,20 @@ class LayerCache:
     def __init__(self, cfg: abi.arkv_cfg, device):
         R, D = cfg.batch * cfg.hkv, cfg.head_dim
         co, cq = cfg.cap_bf16, cfg.cap_fp8
-        i32, f32, u8 = torch.int32, torch.float32, torch.uint8
+        i32, f32, f64, u8 = torch.int32, torch.float32, torch.float64, torch.uint8
         self.cfg = cfg
         self.k16 = torch.zeros((R, co, D), dtype=torch.bfloat16, device=device)
         self.v16 = torch.zeros((R, co, D), dtype=torch.bfloat16, device=device)
         self.pos16 = torch.zeros((R, co), dtype=i32, device=device)
-        self.mu16 = torch.zeros((R, co), dtype=f32, device=device)
-        self.m2_16 = torch.zeros((R, co), dtype=f32, device=device)
+        self.mu16 = torch.zeros((R, co), dtype=f64, device=device)
+        self.m2_16 = torch.zeros((R, co), dtype=f64, device=device)
         self.k8 = torch.zeros((R, cq, D), dtype=u8, device=device)
         self.v8 = torch.zeros((R, cq, D), dtype=u8, device=device)
         self.sk = torch.zeros((R, cq), dtype=f32, device=device)
         self.sv = torch.zeros((R, cq), dtype=f32, device=device)
         self.pos8 = torch.zeros((R, cq), dtype=i32, device=device)
-        self.mu8 = torch.zeros((R, cq), dtype=f32, device=device)
-        self.m2_8 = torch.zeros((R, cq), dtype=f32, device=device)
+        self.mu8 = torch.zeros((R, cq), dtype=f64, device=device)
+        self.m2_8 = torch.zeros((R, cq), dtype=f64, device=device)
         self.n_bf16 = torch.zeros((R,), dtype=i32, device=device)
         self.n_fp8 = torch.zeros((R,), dtype=i32, device=device)
         self.status = torch.zeros((1,), dtype=i32, device=device)

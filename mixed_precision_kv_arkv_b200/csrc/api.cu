@@ -56,10 +56,12 @@ int check_cache(const arkv_layer_cache* c) {
         if (!q) return fail(ARKV_EINVAL, "%s has a null buffer", "cache");
     if (!aligned(c->k16, 16) || !aligned(c->v16, 16) || !aligned(c->k8, 16) || !aligned(c->v8, 16))
         return fail(ARKV_EINVAL, "%s: k16, v16, k8, v8 must be 16-byte aligned", "cache");
-    const void* words[] = {c->pos16, c->mu16, c->m2_16, c->sk, c->sv, c->pos8, c->mu8, c->m2_8,
-                           c->n_bf16, c->n_fp8, c->status};
+    const void* words[] = {c->pos16, c->sk, c->sv, c->pos8, c->n_bf16, c->n_fp8, c->status};
     for (const void* q : words)
         if (!aligned(q, 4)) return fail(ARKV_EINVAL, "%s: 4-byte buffers must be 4-byte aligned", "cache");
+    const void* dwords[] = {c->mu16, c->m2_16, c->mu8, c->m2_8};
+    for (const void* q : dwords)
+        if (!aligned(q, 8)) return fail(ARKV_EINVAL, "%s: mu and M2 buffers must be 8-byte aligned", "cache");
     return ARKV_OK;
 }
 
@@ -86,7 +88,7 @@ PrefillWs prefill_ws(const arkv::LayerDims& d, int n_stride) {
     size_t off = 0;
     w.sumx = off;  off = al(off + sizeof(double) * (size_t)d.R * n_stride * 2);
     w.qstat = off; off = al(off + sizeof(double) * (size_t)d.batch * d.hq * d.n_obs * 3);
-    w.keys = off;  off = al(off + sizeof(uint32_t) * (size_t)d.R * n_stride);
+    w.keys = off;  off = al(off + sizeof(uint64_t) * (size_t)d.R * n_stride);
     w.idx = off;   off = al(off + sizeof(int32_t) * (size_t)d.R * n_stride);
     w.total = off;
     return w;
@@ -143,8 +145,8 @@ int arkv_oq_ratio(const double* stats, int32_t layers, double r_bar, float* r_ou
 }
 
 int arkv_prefill_stats(const arkv_cfg* cfg, const uint16_t* q_obs, const uint16_t* k, int32_t n_ctx_max,
-                       const int32_t* ctx_len, double* stats_out, double* query_stats, float* mu0,
-                       float* m2_0, void* ws, size_t ws_bytes, arkv_stream_t stream) {
+                       const int32_t* ctx_len, double* stats_out, double* query_stats, double* mu0,
+                       double* m2_0, void* ws, size_t ws_bytes, arkv_stream_t stream) {
     ARKV_TRY(check_cfg(cfg));
     if (!q_obs || !k || !ctx_len || !stats_out || !mu0 || !m2_0)
         return fail(ARKV_EINVAL, "%s: null argument", "arkv_prefill_stats");
@@ -165,7 +167,7 @@ int arkv_prefill_stats(const arkv_cfg* cfg, const uint16_t* q_obs, const uint16_
 }
 
 int arkv_quantize_pack(const arkv_cfg* cfg, float r, const uint16_t* k, const uint16_t* v, int32_t n_ctx_max,
-                       const int32_t* ctx_len, const float* mu0, const float* m2_0, arkv_layer_cache* cache,
+                       const int32_t* ctx_len, const double* mu0, const double* m2_0, arkv_layer_cache* cache,
                        uint8_t* tier_out, void* ws, size_t ws_bytes, arkv_stream_t stream) {
     ARKV_TRY(check_cfg(cfg));
     ARKV_TRY(check_cache(cache));
@@ -183,7 +185,7 @@ int arkv_quantize_pack(const arkv_cfg* cfg, float r, const uint16_t* k, const ui
     arkv::PackParams p{};
     p.d = d; p.r = r; p.k = k; p.v = v; p.n_stride = n_ctx_max; p.ctx_len = ctx_len; p.mu0 = mu0; p.m2_0 = m2_0;
     p.c = *cache; p.tier_out = tier_out;
-    p.key_ws = (uint32_t*)((char*)ws + w.keys);
+    p.key_ws = (uint64_t*)((char*)ws + w.keys);
     p.idx_ws = (int32_t*)((char*)ws + w.idx);
     const cudaError_t e = arkv::launch_quantize_pack(p, (cudaStream_t)stream);
     return e == cudaSuccess ? ARKV_OK : cuda_fail(e, "arkv_quantize_pack");
@@ -252,7 +254,7 @@ int arkv_reassign(const arkv_cfg* cfg, int32_t step, float r, const int32_t* ctx
     const size_t slots = (size_t)(d.cap_o + d.cap_q);
     const size_t idx_bytes = (slots * 2 * 4 * d.R + 255) & ~(size_t)255;
     p.idx_ws = (int32_t*)ws;
-    p.key_ws = (uint32_t*)((char*)ws + idx_bytes);
+    p.key_ws = (uint64_t*)((char*)ws + idx_bytes);
     const cudaError_t e = arkv::launch_reassign(p, (cudaStream_t)stream);
     return e == cudaSuccess ? ARKV_OK : cuda_fail(e, "arkv_reassign");
 }

@@ -41,15 +41,18 @@ __device__ __forceinline__ int obs_count_after(int pos, int n0, int t, int n_obs
     return pos < n0 ? min(n_obs, n0 - pos) + t + 1 : t - (pos - n0) + 1;
 }
 
-// Order-preserving map of a float to uint32 (larger float -> larger key).
-__device__ __forceinline__ uint32_t float_key(float f) {
-    const uint32_t u = __float_as_uint(f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+// Order-preserving map of a double to uint64 (larger value -> larger key).  A
+// score is never NaN, so every key of a real score is nonzero: 0 is free to mark
+// a non-candidate.
+__device__ __forceinline__ uint64_t double_key(double f) {
+    const uint64_t u = (uint64_t)__double_as_longlong(f);
+    return (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
 }
 
-// S = mu + gamma * (M2 / n), float32, no contraction.
-__device__ __forceinline__ float score_f32(float mu, float m2, int n, float gamma) {
-    return __fadd_rn(mu, __fmul_rn(gamma, __fdiv_rn(m2, (float)n)));
+// S = mu + gamma * (M2 / n) (ARKV 기술요약 §2.나, population variance), float64,
+// each operation rounded on its own (no contraction), as the oracle evaluates it.
+__device__ __forceinline__ double score_f64(double mu, double m2, int n, float gamma) {
+    return __dadd_rn(mu, __dmul_rn((double)gamma, __ddiv_rn(m2, (double)n)));
 }
 
 // Budget counts of one row, float64 with the operations in a fixed order so that
@@ -166,8 +169,8 @@ struct ReassignParams {
     const int32_t* ctx_len;
     arkv_layer_cache c;
     uint8_t* tier_dbg;
-    uint32_t* key_ws;   // [R][cap_o + cap_q] keys (used when they do not fit in shared memory)
-    int32_t* idx_ws;    // [R][cap_o + cap_q] scratch slot lists
+    uint64_t* key_ws;   // [R][cap_o + cap_q] keys (used when they do not fit in shared memory)
+    int32_t* idx_ws;    // [R][2][cap_o + cap_q] scratch slot lists
 };
 size_t reassign_ws_bytes(const LayerDims& d);
 cudaError_t launch_reassign(const ReassignParams& p, cudaStream_t s);
@@ -179,11 +182,11 @@ struct PackParams {
     const uint16_t* v;
     int n_stride;
     const int32_t* ctx_len;
-    const float* mu0;
-    const float* m2_0;
+    const double* mu0;
+    const double* m2_0;
     arkv_layer_cache c;
     uint8_t* tier_out;
-    uint32_t* key_ws;   // [R][n_stride]
+    uint64_t* key_ws;   // [R][n_stride]
     int32_t* idx_ws;    // [R][n_stride]
 };
 cudaError_t launch_quantize_pack(const PackParams& p, cudaStream_t s);
@@ -196,8 +199,8 @@ struct PrefillParams {
     const int32_t* ctx_len;
     double* stats_out;
     double* query_stats;    // [B][Hq][n_obs][3] or null
-    float* mu0;
-    float* m2_0;
+    double* mu0;
+    double* m2_0;
     double* qml;            // ws [B][Hq][n_obs][2]   (max, sum) per query
     double* qstat;          // ws [B][Hq][n_obs][3]
     double* sumx;           // ws [R][n_stride][2]    (sum x, sum x^2) per key

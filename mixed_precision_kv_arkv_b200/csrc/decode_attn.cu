@@ -61,7 +61,8 @@ struct Smem {
     static constexpr int kL = kM + 16 * 4;                              // float [4][4]
     static constexpr int kRed = kL + 16 * 4;                            // float [4][4]
     static constexpr int kMax = kRed + 16 * 4;                          // float [4]
-    static constexpr int kBytes = kMax + 16 + 1024;                     // + alignment slack
+    static constexpr int kAbort = kMax + 16;                            // int: a wait gave up
+    static constexpr int kBytes = kAbort + 16 + 1024;                   // + alignment slack
     static constexpr int kO = 0;                                        // float [4][4][D], in the idle ring
     static_assert(4 * 4 * D * 4 <= kRing, "the epilogue buffer must fit in the ring");
 };
@@ -414,11 +415,13 @@ __global__ void __launch_bounds__(32 * kWarps) decode_attn_kernel(const __grid_c
         }
         if (tid == 0) {
             p.c.pos16[sl] = p.ctx_len[b] + p.step;
-            p.c.mu16[sl] = 0.f;
-            p.c.m2_16[sl] = 0.f;
+            p.c.mu16[sl] = 0.0;
+            p.c.m2_16[sl] = 0.0;
         }
         asm volatile("fence.proxy.async.global;" ::: "memory");
     }
+    int* sm_abort = reinterpret_cast<int*>(smem + SL::kAbort);
+    if (tid == 0) *sm_abort = 0;
     __syncthreads();
 
     // this warp's tiles: s0 + 16 (warp + 4 i)
@@ -473,8 +476,14 @@ __global__ void __launch_bounds__(32 * kWarps) decode_attn_kernel(const __grid_c
         const int st = i % kStages;
         const int t0 = first + 16 * kWarps * i;
         if (!mbar_wait(&bars[st], (uint32_t)((i / kStages) & 1))) {
-            if (lane == 0) atomicOr(p.c.status, ARKV_STATUS_TIMEOUT);
-            for (int j = i + 1; j < min(i + kStages, ntiles); ++j)   // let issued copies land
+            // a copy did not land in time: flag it, give every copy this warp issued
+            // (this one included) a last bounded chance to land, and leave the ring
+            // alone from here on (the epilogue below does not reuse it)
+            if (lane == 0) {
+                atomicOr(p.c.status, ARKV_STATUS_TIMEOUT);
+                atomicExch(sm_abort, 1);
+            }
+            for (int j = i; j < min(i + kStages, ntiles); ++j)
                 mbar_wait(&bars[j % kStages], (uint32_t)((j / kStages) & 1));
             break;
         }
@@ -500,6 +509,17 @@ __global__ void __launch_bounds__(32 * kWarps) decode_attn_kernel(const __grid_c
     }
 
     __syncthreads();   // every warp has drained its ring: the epilogue may reuse it
+    const size_t pb = (size_t)row * nsplit + split;
+    if (*sm_abort) {
+        // a wait gave up: copies may still be landing in the ring, so write an empty
+        // partial (weight 0 in the merge) without touching shared memory; the status
+        // bit already tells the caller that this call's output is not to be used
+        for (int idx = tid; idx < 4 * D; idx += blockDim.x) {
+            p.part_o[(pb * 4 + idx / D) * D + idx % D] = 0.f;
+            if (idx % D == 0) p.part_ml[pb * 4 + idx / D] = make_float2(kNegInf, 0.f);
+        }
+        return;
+    }
     float (*sm_o)[4][D] = reinterpret_cast<float (*)[4][D]>(smem + SL::kO);
     float (*sm_m)[4] = reinterpret_cast<float (*)[4]>(smem + SL::kM);
     float (*sm_l)[4] = reinterpret_cast<float (*)[4]>(smem + SL::kL);
@@ -544,7 +564,6 @@ __global__ void __launch_bounds__(32 * kWarps) decode_attn_kernel(const __grid_c
         if (w == 0) sm_max[h] = M;
     }
     __syncthreads();
-    const size_t pb = (size_t)row * nsplit + split;
     for (int idx = tid; idx < 4 * D; idx += blockDim.x) {
         const int h = idx / D, dd = idx - h * D;
         float O = 0.f;
@@ -564,7 +583,10 @@ __global__ void __launch_bounds__(32 * kWarps) decode_attn_kernel(const __grid_c
 // L = sum of l_s exp((m_s - M)/sqrt(D)), o = sum of o_s exp(..) / L.  4 x D
 // threads: thread (q, d) sums the splits s = q mod 4 of output dim d, so every
 // thread has only a few independent loads in flight.  Also publishes (M, L) for
-// the score update and advances the row's bf16 count past the appended token.
+// the score update.  The row's bf16 count is advanced past the appended token by
+// the last of the row's G merge CTAs to finish (a ticket in the workspace): every
+// merge CTA of the row reads the count it was launched with, so it may only move
+// once all of them have read it.
 template <int D>
 __global__ void __launch_bounds__(4 * D) merge_kernel(const AttnParams p) {
     const LayerDims& d = p.d;
@@ -646,9 +668,13 @@ __global__ void __launch_bounds__(4 * D) merge_kernel(const AttnParams p) {
         const float o = (sm_acc[dd] + sm_acc[D + dd]) + (sm_acc[2 * D + dd] + sm_acc[3 * D + dd]);
         p.o[((size_t)b * d.hq + g * d.G + h) * D + dd] = o / sm_ML[1];
     }
-    if (h == 0 && tid == 0) {
-        if (n16_old < d.cap_o) p.c.n_bf16[row] = n16_old + 1;
-        else atomicOr(p.c.status, ARKV_STATUS_BF16_FULL);   // the new token was dropped
+    if (tid == 0) {
+        __threadfence();                                 // this CTA's reads of the count come first
+        if (atomicAdd(&p.counter[row], 1u) == (unsigned)(d.G - 1)) {
+            p.counter[row] = 0u;                         // ready for the next call
+            if (n16_old < d.cap_o) p.c.n_bf16[row] = n16_old + 1;
+            else atomicOr(p.c.status, ARKV_STATUS_BF16_FULL);   // the new token was dropped
+        }
     }
 }
 
@@ -669,9 +695,9 @@ __global__ void __launch_bounds__(256) score_update_kernel(const ScoreParams p) 
     const float4 lg = __ldg(bf ? reinterpret_cast<const float4*>(p.logit16) + sl
                                : reinterpret_cast<const float4*>(p.logit8) + sl);
     const int pos = __ldg(bf ? p.c.pos16 + sl : p.c.pos8 + sl);
-    float* __restrict__ mu = bf ? p.c.mu16 + sl : p.c.mu8 + sl;
-    float* __restrict__ m2 = bf ? p.c.m2_16 + sl : p.c.m2_8 + sl;
-    const float mu_old = *mu, m2_old = *m2;
+    double* __restrict__ mu = bf ? p.c.mu16 + sl : p.c.mu8 + sl;
+    double* __restrict__ m2 = bf ? p.c.m2_16 + sl : p.c.m2_8 + sl;
+    const double mu_old = *mu, m2_old = *m2;
     const float lv[4] = {lg.x, lg.y, lg.z, lg.w};
     double x = 0.0;
 #pragma unroll
@@ -682,8 +708,8 @@ __global__ void __launch_bounds__(256) score_update_kernel(const ScoreParams p) 
     const double dl = x - mv;
     mv += dl / (double)n;
     qv += dl * (x - mv);
-    *mu = (float)mv;
-    *m2 = (float)qv;
+    *mu = mv;
+    *m2 = qv;
 }
 
 // ------------------------------------------------------------------ tensor maps

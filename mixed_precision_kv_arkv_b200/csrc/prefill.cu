@@ -219,8 +219,8 @@ __global__ void prefill_welford_kernel(const PrefillParams p) {
         const double sx = sumx[(size_t)k * 2], sx2 = sumx[(size_t)k * 2 + 1];
         const double mu = sx / cnt;
         const double m2 = fmax(sx2 - sx * mu, 0.0);
-        p.mu0[(size_t)row * p.n_stride + k] = (float)mu;
-        p.m2_0[(size_t)row * p.n_stride + k] = (float)m2;
+        p.mu0[(size_t)row * p.n_stride + k] = mu;
+        p.m2_0[(size_t)row * p.n_stride + k] = m2;
     }
 }
 

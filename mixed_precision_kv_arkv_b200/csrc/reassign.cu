@@ -2,12 +2,12 @@
 // under a memory budget with a protected window of the W newest tokens).
 //
 // One 1024-thread CTA per row.  Candidate tokens (live tokens older than the
-// window) get a 32-bit order-preserving key of their score S = mu + gamma*M2/n
-// (0 marks a non-candidate).  Two MSB-first radix selections (8-bit digits,
-// shared-memory histograms) find the n_sel-th best candidate and the n_o-th best
-// kept bf16 token; equal scores are ordered by position through a second radix
-// pass on the position.  The keys live in shared memory when they fit, otherwise
-// in a global workspace (L2-resident).
+// window) get a 64-bit order-preserving key of their float64 score
+// S = mu + gamma*M2/n (0 marks a non-candidate).  Two MSB-first radix selections
+// (8-bit digits, shared-memory histograms) find the n_sel-th best candidate and
+// the n_o-th best kept bf16 token; equal scores are ordered by position through a
+// second radix pass on the position.  The keys live in shared memory when they
+// fit, otherwise in a global workspace (L2-resident).
 //
 // Compaction is in place: in each segment the survivors that sit above the new
 // live count move into the vacated slots below it (k-th source -> k-th hole, both
@@ -21,7 +21,7 @@ namespace arkv {
 
 namespace {
 
-constexpr int kSmemKeyLimit = 48 * 1024;   // keys kept in shared memory up to this many slots
+constexpr int kSmemKeyLimit = 24 * 1024;   // 8-byte keys kept in shared memory up to this many slots
 
 struct RowShared {
     unsigned hist[256];
@@ -100,28 +100,29 @@ __device__ int block_count(int begin, int end, Pred pred, RowShared& sh) {
 // ascending).  Element i is selected iff key(i) > cut, or key(i) == cut and
 // (all_ties or pos(i) <= pos_max).
 struct Sel {
-    uint32_t cut;
+    uint64_t cut;
     int all_ties;
     int pos_max;
 };
 
-__device__ __forceinline__ bool sel_in(const Sel& s, uint32_t key, int pos) {
+__device__ __forceinline__ bool sel_in(const Sel& s, uint64_t key, int pos) {
     return key > s.cut || (key == s.cut && (s.all_ties || pos <= s.pos_max));
 }
 
-// k-th largest key among eligible elements (1 <= k <= count): returns cut and,
-// through need/eq, how many of the elements equal to cut are taken / exist.
-template <class KeyF, class Elig>
-__device__ uint32_t radix_kth(KeyF key, Elig elig, int n, int k, int* need, int* eq, RowShared& sh) {
-    uint32_t prefix = 0, pmask = 0;
+// k-th largest key (of unsigned type KT) among eligible elements (1 <= k <= count):
+// returns cut and, through need/eq, how many of the elements equal to cut are
+// taken / exist.
+template <class KT, class KeyF, class Elig>
+__device__ KT radix_kth(KeyF key, Elig elig, int n, int k, int* need, int* eq, RowShared& sh) {
+    KT prefix = 0, pmask = 0;
     int kk = k, last_eq = 0;
-    for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int shift = 8 * (int)sizeof(KT) - 8; shift >= 0; shift -= 8) {
         for (int i = threadIdx.x; i < 256; i += blockDim.x) sh.hist[i] = 0;
         __syncthreads();
         for (int i = threadIdx.x; i < n; i += blockDim.x) {
             if (!elig(i)) continue;
-            const uint32_t kv = key(i);
-            if ((kv & pmask) == prefix) atomicAdd(&sh.hist[(kv >> shift) & 255u], 1u);
+            const KT kv = key(i);
+            if ((kv & pmask) == prefix) atomicAdd(&sh.hist[(unsigned)(kv >> shift) & 255u], 1u);
         }
         __syncthreads();
         if (threadIdx.x < 32) {
@@ -154,11 +155,11 @@ __device__ uint32_t radix_kth(KeyF key, Elig elig, int n, int k, int* need, int*
             }
         }
         __syncthreads();
-        const uint32_t bin = (uint32_t)sh.sel[0];
+        const KT bin = (KT)sh.sel[0];
         kk -= sh.sel[1];
         last_eq = sh.sel[2];
         prefix |= bin << shift;
-        pmask |= 0xffu << shift;
+        pmask |= (KT)0xff << shift;
         __syncthreads();
     }
     *need = kk;
@@ -171,23 +172,23 @@ template <class KeyF, class PosF, class Elig>
 __device__ Sel select_best(KeyF key, PosF pos, Elig elig, int n, int k, int n_elig, RowShared& sh) {
     Sel s;
     if (k <= 0) {
-        s.cut = 0xffffffffu; s.all_ties = 0; s.pos_max = -1;
+        s.cut = ~0ull; s.all_ties = 0; s.pos_max = -1;
         return s;
     }
     if (k >= n_elig) {
-        s.cut = 0u; s.all_ties = 1; s.pos_max = 0;
+        s.cut = 0ull; s.all_ties = 1; s.pos_max = 0;
         return s;
     }
     int need, eq;
-    s.cut = radix_kth(key, elig, n, k, &need, &eq, sh);
+    s.cut = radix_kth<uint64_t>(key, elig, n, k, &need, &eq, sh);
     s.all_ties = need >= eq;
     s.pos_max = 0;
     if (!s.all_ties) {
-        const uint32_t cut = s.cut;
+        const uint64_t cut = s.cut;
         int need2, eq2;
-        const uint32_t c2 = radix_kth([&](int i) { return ~(uint32_t)pos(i); },
-                                      [&](int i) { return elig(i) && key(i) == cut; }, n, need,
-                                      &need2, &eq2, sh);
+        const uint32_t c2 = radix_kth<uint32_t>([&](int i) { return ~(uint32_t)pos(i); },
+                                                [&](int i) { return elig(i) && key(i) == cut; }, n, need,
+                                                &need2, &eq2, sh);
         s.pos_max = (int)~c2;
     }
     return s;
@@ -227,7 +228,7 @@ __device__ __forceinline__ float warp_quantize_row(const uint16_t* src, uint8_t*
 
 // ------------------------------------------------------------------ reassignment
 // Slot outcomes, frozen before any data moves.
-constexpr uint32_t kStayBf16 = 0, kDemote = 1, kEvict = 2, kStayFp8 = 3;
+constexpr uint64_t kStayBf16 = 0, kDemote = 1, kEvict = 2, kStayFp8 = 3;
 
 template <int D>
 __global__ void __launch_bounds__(kRowThreads) reassign_kernel(const ReassignParams p) {
@@ -235,7 +236,7 @@ __global__ void __launch_bounds__(kRowThreads) reassign_kernel(const ReassignPar
     const int row = blockIdx.x, b = row / d.hkv;
     const int tid = threadIdx.x, warp = tid >> 5, nwarps = blockDim.x >> 5;
     __shared__ RowShared sh;
-    extern __shared__ uint32_t sm_keys[];
+    extern __shared__ uint64_t sm_keys[];
 
     const int n16 = min(max(p.c.n_bf16[row], 0), d.cap_o);
     const int n8 = min(max(p.c.n_fp8[row], 0), d.cap_q);
@@ -245,7 +246,7 @@ __global__ void __launch_bounds__(kRowThreads) reassign_kernel(const ReassignPar
     const int winlo = nt - d.W;
     const size_t slots = (size_t)(d.cap_o + d.cap_q);
     const size_t b16 = (size_t)row * d.cap_o, b8 = (size_t)row * d.cap_q;
-    uint32_t* keys = (slots <= (size_t)kSmemKeyLimit) ? sm_keys : p.key_ws + (size_t)row * slots;
+    uint64_t* keys = (slots <= (size_t)kSmemKeyLimit) ? sm_keys : p.key_ws + (size_t)row * slots;
     int32_t* src_list = p.idx_ws + (size_t)row * 2 * slots;   // [slots]
     int32_t* hole_list = src_list + slots;                    // [slots]
 
@@ -257,11 +258,11 @@ __global__ void __launch_bounds__(kRowThreads) reassign_kernel(const ReassignPar
         const bool bf = i < n16;
         const size_t sl = bf ? b16 + i : b8 + (i - n16);
         const int pos = bf ? p.c.pos16[sl] : p.c.pos8[sl];
-        uint32_t key = 0;
+        uint64_t key = 0;
         if (!bf || pos < winlo) {
-            const float mu = bf ? p.c.mu16[sl] : p.c.mu8[sl];
-            const float m2 = bf ? p.c.m2_16[sl] : p.c.m2_8[sl];
-            key = float_key(score_f32(mu, m2, obs_count_after(pos, n0, p.step, d.n_obs), d.gamma));
+            const double mu = bf ? p.c.mu16[sl] : p.c.mu8[sl];
+            const double m2 = bf ? p.c.m2_16[sl] : p.c.m2_8[sl];
+            key = double_key(score_f64(mu, m2, obs_count_after(pos, n0, p.step, d.n_obs), d.gamma));
             ++ncand;
         }
         keys[i] = key;
@@ -276,11 +277,11 @@ __global__ void __launch_bounds__(kRowThreads) reassign_kernel(const ReassignPar
     __syncthreads();
     const int n_sel = sh.misc[0], n_o = sh.misc[1];
 
-    auto keyf = [&](int i) -> uint32_t { return keys[i]; };
+    auto keyf = [&](int i) -> uint64_t { return keys[i]; };
     const Sel keep = select_best(keyf, pos_of, [&](int i) { return keys[i] != 0u; }, n, n_sel,
                                  ncand, sh);
     auto kept = [&](int i) -> bool {
-        const uint32_t k = keys[i];
+        const uint64_t k = keys[i];
         return k != 0u && sel_in(keep, k, k == keep.cut ? pos_of(i) : 0);
     };
     auto kept16 = [&](int i) -> bool { return i < n16 && kept(i); };
@@ -289,8 +290,8 @@ __global__ void __launch_bounds__(kRowThreads) reassign_kernel(const ReassignPar
 
     // freeze the outcome of every slot
     for (int i = tid; i < n; i += blockDim.x) {
-        const uint32_t k = keys[i];
-        uint32_t st;
+        const uint64_t k = keys[i];
+        uint64_t st;
         if (i < n16) {
             if (k == 0u) {
                 st = kStayBf16;   // window
@@ -318,11 +319,13 @@ __global__ void __launch_bounds__(kRowThreads) reassign_kernel(const ReassignPar
     }
     const int n8_new = n8_stay + n_dem;
 
-    if (p.tier_dbg) {
-        uint8_t* td = p.tier_dbg + (size_t)row * slots;
+    // debug tiers: demotions are reported where they are enumerated below (the ones
+    // past the fp8 capacity become evictions)
+    uint8_t* td = p.tier_dbg ? p.tier_dbg + (size_t)row * slots : nullptr;
+    if (td) {
         for (int i = tid; i < n16; i += blockDim.x) {
-            const uint32_t st = keys[i];
-            td[i] = st == kStayBf16 ? ARKV_TIER_ORIGINAL : (st == kDemote ? ARKV_TIER_QUANTIZED : ARKV_TIER_EVICTED);
+            const uint64_t st = keys[i];
+            if (st != kDemote) td[i] = st == kStayBf16 ? ARKV_TIER_ORIGINAL : ARKV_TIER_EVICTED;
         }
         for (int j = tid; j < n8; j += blockDim.x)
             td[d.cap_o + j] = keys[n16 + j] == kStayFp8 ? ARKV_TIER_QUANTIZED : ARKV_TIER_EVICTED;
@@ -349,7 +352,10 @@ __global__ void __launch_bounds__(kRowThreads) reassign_kernel(const ReassignPar
         }
     }
     __syncthreads();
-    block_enumerate(0, n16, is_demote, [&](int i, int r) { src_list[r] = i; }, sh);
+    block_enumerate(0, n16, is_demote, [&](int i, int r) {
+        src_list[r] = i;
+        if (td) td[i] = r < n_dem ? ARKV_TIER_QUANTIZED : ARKV_TIER_EVICTED;
+    }, sh);
     __syncthreads();
     for (int r = warp; r < n_dem; r += nwarps) {
         const int src = src_list[r], dst = hole_list[n_mov8 + r];
@@ -395,21 +401,21 @@ __global__ void __launch_bounds__(kRowThreads) pack_kernel(const PackParams p) {
     const int row = blockIdx.x, b = row / d.hkv, g = row - b * d.hkv;
     const int tid = threadIdx.x, warp = tid >> 5, nwarps = blockDim.x >> 5;
     __shared__ RowShared sh;
-    extern __shared__ uint32_t sm_keys[];
+    extern __shared__ uint64_t sm_keys[];
 
     const int n0 = min(p.ctx_len[b], p.n_stride);
     const int winlo = n0 - d.W;
     const size_t src_row = ((size_t)b * d.hkv + g) * p.n_stride;
     const size_t b16 = (size_t)row * d.cap_o, b8 = (size_t)row * d.cap_q;
-    uint32_t* keys = (p.n_stride <= kSmemKeyLimit) ? sm_keys : p.key_ws + (size_t)row * p.n_stride;
+    uint64_t* keys = (p.n_stride <= kSmemKeyLimit) ? sm_keys : p.key_ws + (size_t)row * p.n_stride;
     int32_t* rank = p.idx_ws + (size_t)row * p.n_stride;
 
     int ncand = 0;
     for (int i = tid; i < n0; i += blockDim.x) {
-        uint32_t key = 0;
+        uint64_t key = 0;
         if (i < winlo) {
-            key = float_key(score_f32(p.mu0[src_row + i], p.m2_0[src_row + i],
-                                      obs_count_after(i, n0, -1, d.n_obs), d.gamma));
+            key = double_key(score_f64(p.mu0[src_row + i], p.m2_0[src_row + i],
+                                       obs_count_after(i, n0, -1, d.n_obs), d.gamma));
             ++ncand;
         }
         keys[i] = key;
@@ -423,7 +429,7 @@ __global__ void __launch_bounds__(kRowThreads) pack_kernel(const PackParams p) {
     }
     __syncthreads();
     const int n_sel = sh.misc[0], n_o = sh.misc[1];
-    auto keyf = [&](int i) -> uint32_t { return keys[i]; };
+    auto keyf = [&](int i) -> uint64_t { return keys[i]; };
     auto posf = [&](int i) -> int { return i; };
     const Sel keep = select_best(keyf, posf, [&](int i) { return keys[i] != 0u; }, n0, n_sel, ncand, sh);
     auto kept = [&](int i) -> bool { return keys[i] != 0u && sel_in(keep, keys[i], i); };
@@ -444,7 +450,7 @@ __global__ void __launch_bounds__(kRowThreads) pack_kernel(const PackParams p) {
             to[i] = is_o(i) ? ARKV_TIER_ORIGINAL : (is_q(i) ? ARKV_TIER_QUANTIZED : ARKV_TIER_EVICTED);
     }
     for (int i = warp; i < n0; i += nwarps) {
-        const uint32_t k = keys[i];
+        const uint64_t k = keys[i];
         const bool o = k == 0u || (k != 0u && sel_in(keep, k, i) && sel_in(orig, k, i));
         const bool q = !o && k != 0u && sel_in(keep, k, i);
         if (!o && !q) continue;
@@ -499,13 +505,13 @@ unsigned char g_smem_reassign128[64], g_smem_reassign64[64], g_smem_pack128[64],
 
 size_t reassign_ws_bytes(const LayerDims& d) {
     const size_t per_row = (size_t)(d.cap_o + d.cap_q);
-    const size_t keys = (d.cap_o + d.cap_q <= kSmemKeyLimit) ? 0 : per_row * 4 * d.R;
-    return ((keys + 255) & ~(size_t)255) + per_row * 2 * 4 * d.R + 256;
+    const size_t keys = (d.cap_o + d.cap_q <= kSmemKeyLimit) ? 0 : per_row * 8 * d.R;
+    return ((per_row * 2 * 4 * d.R + 255) & ~(size_t)255) + keys + 256;
 }
 
 cudaError_t launch_reassign(const ReassignParams& p, cudaStream_t s) {
     const size_t slots = (size_t)(p.d.cap_o + p.d.cap_q);
-    const size_t dyn = slots <= (size_t)kSmemKeyLimit ? slots * 4 : 0;
+    const size_t dyn = slots <= (size_t)kSmemKeyLimit ? slots * 8 : 0;
     cudaError_t e;
     if (p.d.D == 128) {
         e = allow_max_dyn_smem(reassign_kernel<128>, g_smem_reassign128);
@@ -520,7 +526,7 @@ cudaError_t launch_reassign(const ReassignParams& p, cudaStream_t s) {
 }
 
 cudaError_t launch_quantize_pack(const PackParams& p, cudaStream_t s) {
-    const size_t dyn = p.n_stride <= kSmemKeyLimit ? (size_t)p.n_stride * 4 : 0;
+    const size_t dyn = p.n_stride <= kSmemKeyLimit ? (size_t)p.n_stride * 8 : 0;
     cudaError_t e;
     if (p.d.D == 128) {
         e = allow_max_dyn_smem(pack_kernel<128>, g_smem_pack128);

@@ -11,7 +11,8 @@
 // lives in g_noalloc_scratch below.
 //
 // The array is a module global, so every GPU that loads this library holds
-// ARKV_NOALLOC_SCRATCH_BYTES of it until the process exits.  All calls share it
+// ARKV_NOALLOC_SCRATCH_BYTES of it until the process exits (or its context is
+// destroyed, after which the next call finds the array's new address).  All calls share it
 // and it keeps whatever the last call left; the kernel writes every scratch word
 // before it reads it, so nothing needs clearing.  Calls whose executions overlap
 // on the GPU (different streams, or different layers without ordering) race on
@@ -20,6 +21,8 @@
 
 #include <mutex>
 
+#include <cudaTypedefs.h>
+
 #include "arkv_internal.cuh"
 
 namespace {
@@ -27,24 +30,53 @@ namespace {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[ARKV_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices];
-std::once_flag g_scratch_once[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
+unsigned long long g_scratch_ctx[kMaxDevices];   // id of the context the address belongs to
+bool g_scratch_set[kMaxDevices];
+
+// Unique id of the calling thread's current CUDA context (driver entry points,
+// looked up once), or 0 if it cannot be had.
+unsigned long long current_context_id() {
+    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx) get_id(ctx, &id);
+    return id;
+}
 
 // The device address of g_noalloc_scratch on the current device.  In host code
-// the array's name is only a host-side handle, so the address is looked up once
-// per device (with that device current) and cached.
+// the array's name is only a host-side handle, so the address is looked up with
+// the device current (cudaGetSymbolAddress) the first time, and again whenever
+// the device's context has changed since (the module, and with it the array, is
+// reloaded in a new context).
 cudaError_t scratch_address(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::call_once(g_scratch_once[dev], [dev] {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    const unsigned long long ctx = current_context_id();
+    if (!g_scratch_set[dev] || (ctx != 0 && ctx != g_scratch_ctx[dev])) {
         void* p = nullptr;
-        g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
         g_scratch_ptr[dev] = p;
-    });
-    if (g_scratch_err[dev] != cudaSuccess) return g_scratch_err[dev];
+        g_scratch_ctx[dev] = current_context_id();   // the lookup made the context current if it was not
+        g_scratch_set[dev] = true;
+    }
     *out = g_scratch_ptr[dev];
     return cudaSuccess;
 }

@@ -46,15 +46,15 @@ def upload_rows(lay: A.OracleLayer, cache: LayerCache, rows=None):
         cache.k16[rid, :no] = bits_to_bf16_tensor(inputs.round_bf16(row.kf[o]), dev)
         cache.v16[rid, :no] = bits_to_bf16_tensor(inputs.round_bf16(row.vf[o]), dev)
         cache.pos16[rid, :no] = torch.from_numpy(row.pos[o].astype(np.int32)).to(dev)
-        cache.mu16[rid, :no] = torch.from_numpy(row.mu[o].astype(np.float32)).to(dev)
-        cache.m2_16[rid, :no] = torch.from_numpy(row.m2[o].astype(np.float32)).to(dev)
+        cache.mu16[rid, :no] = torch.from_numpy(row.mu[o].astype(np.float64)).to(dev)
+        cache.m2_16[rid, :no] = torch.from_numpy(row.m2[o].astype(np.float64)).to(dev)
         cache.k8[rid, :nq] = torch.from_numpy(row.kc[q]).to(dev)
         cache.v8[rid, :nq] = torch.from_numpy(row.vc[q]).to(dev)
         cache.sk[rid, :nq] = torch.from_numpy(row.sk[q]).to(dev)
         cache.sv[rid, :nq] = torch.from_numpy(row.sv[q]).to(dev)
         cache.pos8[rid, :nq] = torch.from_numpy(row.pos[q].astype(np.int32)).to(dev)
-        cache.mu8[rid, :nq] = torch.from_numpy(row.mu[q].astype(np.float32)).to(dev)
-        cache.m2_8[rid, :nq] = torch.from_numpy(row.m2[q].astype(np.float32)).to(dev)
+        cache.mu8[rid, :nq] = torch.from_numpy(row.mu[q].astype(np.float64)).to(dev)
+        cache.m2_8[rid, :nq] = torch.from_numpy(row.m2[q].astype(np.float64)).to(dev)
         cache.n_bf16[rid] = no
         cache.n_fp8[rid] = nq
 
@@ -79,8 +79,8 @@ def download_row(cache: LayerCache, rid: int) -> dict:
         "k16": kb, "v16": vb, "kc": kc, "vc": vc,
         "sk": np.concatenate([np.ones(n16, np.float32), g(cache.sk, n8)])[order],
         "sv": np.concatenate([np.ones(n16, np.float32), g(cache.sv, n8)])[order],
-        "mu": np.concatenate([g(cache.mu16, n16), g(cache.mu8, n8)]).astype(np.float64)[order],
-        "m2": np.concatenate([g(cache.m2_16, n16), g(cache.m2_8, n8)]).astype(np.float64)[order],
+        "mu": np.concatenate([g(cache.mu16, n16), g(cache.mu8, n8)])[order],
+        "m2": np.concatenate([g(cache.m2_16, n16), g(cache.m2_8, n8)])[order],
         "slots": np.concatenate([np.arange(n16), cache.cfg.cap_bf16 + np.arange(n8)])[order],
     }
 
@@ -160,8 +160,8 @@ class DeviceLayer:
         """arkv_prefill_stats + arkv_quantize_pack on torch device tensors."""
         wl, dev = self.wl, self.device
         R, N = wl.rows, self.n_stride
-        self.mu0 = torch.zeros((R, N), dtype=torch.float32, device=dev)
-        self.m2_0 = torch.zeros((R, N), dtype=torch.float32, device=dev)
+        self.mu0 = torch.zeros((R, N), dtype=torch.float64, device=dev)
+        self.m2_0 = torch.zeros((R, N), dtype=torch.float64, device=dev)
         self.stats = torch.zeros(3, dtype=torch.float64, device=dev)
         self.qstats = torch.zeros((wl.batch, wl.hq, wl.n_obs, 3), dtype=torch.float64, device=dev)
         abi.arkv_prefill_stats(self.cfg, q_obs.data_ptr(), k.data_ptr(), N, ctx_len.data_ptr(),

@@ -97,8 +97,8 @@ def run_scenario(wl, steps, dev, rows=None, r=None, kernel_parity=False, seed=0,
     m20 = torch.zeros_like(dl.m2_0)
     for rid in rows:
         row = lay.rows[rid]
-        mu0[rid, :len(row.mu)] = torch.from_numpy(row.mu.astype(np.float32)).to(dev)
-        m20[rid, :len(row.m2)] = torch.from_numpy(row.m2.astype(np.float32)).to(dev)
+        mu0[rid, :len(row.mu)] = torch.from_numpy(row.mu.astype(np.float64)).to(dev)
+        m20[rid, :len(row.m2)] = torch.from_numpy(row.m2.astype(np.float64)).to(dev)
     dl.pack(k_t, v_t, ctx_t, r, mu0, m20)
     recs = lay.initial_reassign(r)
     tier_out = dl.tier_out.cpu().numpy()
@@ -118,6 +118,8 @@ def run_scenario(wl, steps, dev, rows=None, r=None, kernel_parity=False, seed=0,
     assert int(dl.cache.status.item()) == 0
 
     o = torch.zeros((wl.batch, wl.hq, wl.head_dim), dtype=torch.float32, device=dev)
+    summary["log"] = []                     # one record per reassignment interval
+    iv = {"o_rel": 0.0, "s_rel": 0.0}
     for t in range(steps):
         if kernel_parity:
             H.upload_rows(lay, dl.cache, rows)
@@ -129,12 +131,15 @@ def run_scenario(wl, steps, dev, rows=None, r=None, kernel_parity=False, seed=0,
         for rid in rows:
             b, g = divmod(rid, wl.hkv)
             sl = slice(g * wl.group, (g + 1) * wl.group)
-            summary["o_rel"] = max(summary["o_rel"], H.max_rel_per_row(og[b, sl], o_ref[b, sl]))
+            iv["o_rel"] = max(iv["o_rel"], H.max_rel_per_row(og[b, sl], o_ref[b, sl]))
             gpu = H.download_row(dl.cache, rid)
-            summary["s_rel"] = max(summary["s_rel"], H.score_rel_err(gpu, lay.rows[rid], wl.gamma))
+            iv["s_rel"] = max(iv["s_rel"], H.score_rel_err(gpu, lay.rows[rid], wl.gamma))
+        summary["o_rel"] = max(summary["o_rel"], iv["o_rel"])
+        summary["s_rel"] = max(summary["s_rel"], iv["s_rel"])
         assert summary["o_rel"] <= O_TOL, (t, summary)
         assert summary["s_rel"] <= S_TOL, (t, summary)
         if (t + 1) % wl.reassign_interval == 0:
+            exempt_before = summary["exempt"]
             pre_rows = {rid: H.download_row(dl.cache, rid) for rid in rows}
             recs = lay.reassign(t, r)
             dl.reassign(t, r, ctx_t)
@@ -156,6 +161,13 @@ def run_scenario(wl, steps, dev, rows=None, r=None, kernel_parity=False, seed=0,
                 win = gpu["pos"] >= n_t - wl.window
                 assert win.sum() == wl.window and gpu["orig"][win].all()
             assert int(dl.cache.status.item()) == 0
+            rec = {"step": t, "o_rel": iv["o_rel"], "s_rel": iv["s_rel"],
+                   "exempt": summary["exempt"] - exempt_before,
+                   "tokens": sum(len(recs[rid]["pos"]) for rid in rows)}
+            summary["log"].append(rec)
+            print(f"PARITY {wl.name} rows={list(rows)} " + " ".join(f"{k}={v:.3g}" if isinstance(v, float)
+                                                                 else f"{k}={v}" for k, v in rec.items()))
+            iv = {"o_rel": 0.0, "s_rel": 0.0}
     if summary["tokens"]:
         assert summary["exempt"] <= exempt_budget * summary["tokens"] + 2, summary
     return summary
@@ -221,8 +233,8 @@ def test_uniform_attention_ties_break_by_position(cuda):
     dl.prefill(k_t, v_t, q_t, ctx_t, r=None)
     mu0, m20 = torch.zeros_like(dl.mu0), torch.zeros_like(dl.m2_0)
     for rid, row in lay.rows.items():
-        mu0[rid, :len(row.mu)] = torch.from_numpy(row.mu.astype(np.float32)).to(cuda)
-        m20[rid, :len(row.m2)] = torch.from_numpy(row.m2.astype(np.float32)).to(cuda)
+        mu0[rid, :len(row.mu)] = torch.from_numpy(row.mu.astype(np.float64)).to(cuda)
+        m20[rid, :len(row.m2)] = torch.from_numpy(row.m2.astype(np.float64)).to(cuda)
     dl.pack(k_t, v_t, ctx_t, 0.5, mu0, m20)
     recs = lay.initial_reassign(0.5)
     tier_out = dl.tier_out.cpu().numpy()
