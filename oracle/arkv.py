@@ -32,7 +32,9 @@ Where the page leaves a step open, the reading taken is named R-<n>:
   R-11 r = n_O / (n_O + n_Q) over the non-window kept tokens
 The FP8 path (scale and code) is float32, as the format fixes it; the budget
 arithmetic is float64 with the operations in the order written, so that any
-implementation doing the same operations obtains the same integers.
+implementation doing the same operations obtains the same integers.  The
+Quantization tier's format is E4M3 unless a caller names E5M2 (the page says
+"FP8", which covers both).
 """
 from __future__ import annotations
 
@@ -41,10 +43,12 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
-from . import e4m3
+from . import e4m3, e5m2
 
 ORIGINAL, QUANTIZED, EVICTED = 0, 1, 2
 E4M3_MAX = np.float32(448.0)
+# the Quantization tier's FP8 formats: codec and largest finite value
+FORMATS = {"e4m3": (e4m3, E4M3_MAX), "e5m2": (e5m2, np.float32(57344.0))}
 
 
 # ------------------------------------------------------------------ sizes (R-8)
@@ -59,22 +63,24 @@ def bytes_quantized(D: int) -> int:
 
 
 # ------------------------------------------------------------------ FP8 (§2.다)
-def quantize_token_head(x: np.ndarray):
-    """Quantize the last axis (one token-head vector) to E4M3 with an absmax scale.
+def quantize_token_head(x: np.ndarray, fmt: str = "e4m3"):
+    """Quantize the last axis (one token-head vector) to FP8 with an absmax scale.
 
-    s = fl32(amax / 448) (s = 1 when amax = 0); code = RNE_E4M3(fl32(x / s)).
+    s = fl32(amax / FMAX) (s = 1 when amax = 0); code = RNE_FP8(fl32(x / s)), with
+    FMAX = 448 for E4M3 and 57344 for E5M2.
     Returns (codes uint8 [..., D], scales float32 [...]).
     """
+    codec, fmax = FORMATS[fmt]
     x32 = np.asarray(x, dtype=np.float32)
     amax = np.max(np.abs(x32), axis=-1)
-    s = np.where(amax == 0, np.float32(1.0), amax / E4M3_MAX).astype(np.float32)
-    codes = e4m3.encode((x32 / s[..., None]).astype(np.float32))
+    s = np.where(amax == 0, np.float32(1.0), amax / fmax).astype(np.float32)
+    codes = codec.encode((x32 / s[..., None]).astype(np.float32))
     return codes, s
 
 
-def dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+def dequantize(codes: np.ndarray, scales: np.ndarray, fmt: str = "e4m3") -> np.ndarray:
     """The dequantized value, code value times its scale, exact in float64."""
-    return e4m3.decode(codes) * np.asarray(scales, np.float64)[..., None]
+    return FORMATS[fmt][0].decode(codes) * np.asarray(scales, np.float64)[..., None]
 
 
 # ------------------------------------------------------------------ attention
@@ -221,15 +227,16 @@ class Row:
     cnt: np.ndarray = None       # Welford count
     mu: np.ndarray = None
     m2: np.ndarray = None
+    fmt: str = "e4m3"            # FP8 format of the Quantized tokens
 
     @staticmethod
-    def from_prefill(K, V, mu, m2, cnt):
+    def from_prefill(K, V, mu, m2, cnt, fmt: str = "e4m3"):
         n, D = K.shape
         return Row(D=D, pos=np.arange(n, dtype=np.int64), orig=np.ones(n, bool),
                    kf=K.copy(), vf=V.copy(), kc=np.zeros((n, D), np.uint8),
                    vc=np.zeros((n, D), np.uint8), sk=np.ones(n, np.float32),
                    sv=np.ones(n, np.float32), cnt=cnt.astype(np.int64).copy(),
-                   mu=mu.copy(), m2=m2.copy())
+                   mu=mu.copy(), m2=m2.copy(), fmt=fmt)
 
     def subset(self, keep):
         for name in ("pos", "orig", "kf", "vf", "kc", "vc", "sk", "sv", "cnt", "mu", "m2"):
@@ -237,8 +244,8 @@ class Row:
 
     def keys_values(self):
         """K and V as attention sees them: bf16 values, or dequantized codes (§2.다)."""
-        Kq = dequantize(self.kc, self.sk)
-        Vq = dequantize(self.vc, self.sv)
+        Kq = dequantize(self.kc, self.sk, self.fmt)
+        Vq = dequantize(self.vc, self.sv, self.fmt)
         o = self.orig[:, None]
         return np.where(o, self.kf, Kq), np.where(o, self.vf, Vq)
 
@@ -288,8 +295,8 @@ def reassign_row(row: Row, n_t: int, W: int, beta: float, r: float, gamma: float
     tiers[cand] = tiers_c
     demote = row.orig & (tiers == QUANTIZED)
     if demote.any():
-        row.kc[demote], row.sk[demote] = quantize_token_head(row.kf[demote])
-        row.vc[demote], row.sv[demote] = quantize_token_head(row.vf[demote])
+        row.kc[demote], row.sk[demote] = quantize_token_head(row.kf[demote], row.fmt)
+        row.vc[demote], row.sv[demote] = quantize_token_head(row.vf[demote], row.fmt)
         row.orig[demote] = False
     rec = {"pos": row.pos.copy(), "tier": tiers, "S": S, "cand": cand, "n_sel": n_sel,
            "n_o": n_o, "cut_keep": cut_keep, "cut_orig": cut_o}
@@ -306,8 +313,9 @@ class OracleLayer:
     subset of row indices (b * Hkv + g).
     """
 
-    def __init__(self, batch, hq, hkv, D, W, n_obs, beta, gamma, ctx_len, rows=None):
+    def __init__(self, batch, hq, hkv, D, W, n_obs, beta, gamma, ctx_len, rows=None, fmt="e4m3"):
         self.B, self.Hq, self.Hkv, self.D = batch, hq, hkv, D
+        self.fmt = fmt
         self.G = hq // hkv
         self.W, self.n_obs, self.beta, self.gamma = W, n_obs, beta, gamma
         self.ctx_len = np.asarray(ctx_len, np.int64)
@@ -323,7 +331,7 @@ class OracleLayer:
             qg = q_obs[b, g * self.G:(g + 1) * self.G]
             st, mu, m2, cnt = prefill_row(qg, k[b, g, :n])
             self.query_stats[rid] = st
-            self.rows[rid] = Row.from_prefill(k[b, g, :n], v[b, g, :n], mu, m2, cnt)
+            self.rows[rid] = Row.from_prefill(k[b, g, :n], v[b, g, :n], mu, m2, cnt, self.fmt)
 
     def layer_stats(self) -> np.ndarray:
         """Mean (H, v, kappa) over every (sequence, query head, observation query)."""

@@ -1,4 +1,4 @@
-"""Compile the oracle's C code (the E4M3 codec) into oracle/liboracle_e4m3.so.
+"""Compile the oracle's C code (the E4M3 and E5M2 codecs) into oracle/liboracle_fp8.so.
 
 Test infrastructure only: see the package docstring.
 """
@@ -7,15 +7,15 @@ import subprocess
 import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-SRC = os.path.join(HERE, "e4m3.c")
-LIB = os.path.join(HERE, "liboracle_e4m3.so")
+SRCS = [os.path.join(HERE, "e4m3.c"), os.path.join(HERE, "e5m2.c")]
+LIB = os.path.join(HERE, "liboracle_fp8.so")
 
 
 def build(force: bool = False) -> str:
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
+    if not force and os.path.exists(LIB) and all(os.path.getmtime(LIB) >= os.path.getmtime(s) for s in SRCS):
         return LIB
     cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
-           "-fno-fast-math", SRC, "-o", LIB, "-lm"]
+           "-fno-fast-math", *SRCS, "-o", LIB, "-lm"]
     subprocess.run(cmd, check=True)
     return LIB
 

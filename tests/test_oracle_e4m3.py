@@ -74,7 +74,11 @@ def test_bits_range_matches_elementwise():
     assert (got == e4m3.encode(x)).all()
 
 
-@pytest.mark.parametrize("exp_bits", [0x00, 0x38, 0x3C, 0x40, 0x43, 0x7F])
+# float32 exponent fields of the binades the format spans: below its smallest
+# subnormal (2^-10), its subnormals (2^-9 .. 2^-7), its smallest normal (2^-6), 1,
+# and its top binades ([128, 256) and [256, 512), where 448 saturates), plus the
+# float32 subnormals
+@pytest.mark.parametrize("exp_bits", [0x00, 0x75, 0x76, 0x77, 0x78, 0x79, 0x7F, 0x86, 0x87])
 def test_exhaustive_mantissa_sweep_against_torch(exp_bits):
     """Every float32 in selected binades (all 2^23 mantissas each), positive and negative."""
     for sign in (0, 1):

@@ -29,6 +29,17 @@ def test_quantize_hand_cases():
     assert list(codes) == [0x71, 0x79, 0x7E]
 
 
+def test_quantize_e5m2_hand_cases():
+    """The second FP8 format: s = fl32(amax / 57344)."""
+    codes, s = A.quantize_token_head(np.array([57344.0, -28672.0, 0.5, 0.0]), "e5m2")
+    assert s == np.float32(1.0)
+    assert list(codes) == [0x7B, 0xF7, 0x38, 0x00]
+    # amax = 3: 1/s = 19114.7 -> 20480 (0x75); 2/s = 38229.3 -> 40960 (0x79); 3/s -> 57344
+    codes, s = A.quantize_token_head(np.array([1.0, 2.0, 3.0]), "e5m2")
+    assert s == np.float32(3.0) / np.float32(57344.0)
+    assert list(codes) == [0x75, 0x79, 0x7B]
+
+
 def test_quantize_error_bound():
     """|x - deq(q(x))| <= half an E4M3 spacing at the scaled magnitude (plus fp32 rounding)."""
     rng = np.random.default_rng(1)
@@ -65,18 +76,19 @@ def test_full_budget_attention_equals_exact_softmax_attention():
     np.testing.assert_allclose(x.sum(), G, rtol=1e-12)
 
 
-def test_mixed_cache_attention_equals_attention_over_dequantized_tensors():
+@pytest.mark.parametrize("fmt,tdtype", [("e4m3", torch.float8_e4m3fn), ("e5m2", torch.float8_e5m2)])
+def test_mixed_cache_attention_equals_attention_over_dequantized_tensors(fmt, tdtype):
     """Brute force from the cache tensors: dequantize with torch's float8 decoder and
     run SDPA; must equal the oracle's attention over the tri-state row."""
     rng = np.random.default_rng(3)
     D, G, N = 16, 2, 50
     K = rng.standard_normal((N, D)); V = rng.standard_normal((N, D))
-    row = A.Row.from_prefill(K, V, np.zeros(N), np.zeros(N), np.ones(N))
+    row = A.Row.from_prefill(K, V, np.zeros(N), np.zeros(N), np.ones(N), fmt)
     qmask = rng.random(N) < 0.5
-    row.kc[qmask], row.sk[qmask] = A.quantize_token_head(K[qmask])
-    row.vc[qmask], row.sv[qmask] = A.quantize_token_head(V[qmask])
+    row.kc[qmask], row.sk[qmask] = A.quantize_token_head(K[qmask], fmt)
+    row.vc[qmask], row.sv[qmask] = A.quantize_token_head(V[qmask], fmt)
     row.orig[qmask] = False
-    f8 = lambda c: torch.from_numpy(c.copy()).view(torch.float8_e4m3fn).double().numpy()
+    f8 = lambda c: torch.from_numpy(c.copy()).view(tdtype).double().numpy()
     Kd = np.where(qmask[:, None], f8(row.kc) * row.sk[:, None].astype(np.float64), K)
     Vd = np.where(qmask[:, None], f8(row.vc) * row.sv[:, None].astype(np.float64), V)
     q = rng.standard_normal((G, D))
