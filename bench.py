@@ -75,10 +75,10 @@ def job_tokens_per_s(batch: int, steps: int, world: int, ms: float) -> float:
     return batch * steps * world / (ms * 1e-3)
 
 
-# kernels one decode step of one layer launches: decode_attn_kernel and merge_kernel
-# (arkv_decode_attn), score_update_kernel (arkv_score_update); arkv_reassign adds
-# reassign_kernel every reassignment interval
-KERNELS_PER_LAYER_STEP = 3
+# kernels one decode step of one layer launches: decode_attn_kernel (arkv_decode_attn,
+# the split merge included) and score_update_kernel (arkv_score_update);
+# arkv_reassign adds reassign_kernel every reassignment interval
+KERNELS_PER_LAYER_STEP = 2
 
 
 def kernel_traffic(kernel_file: str):
@@ -160,7 +160,8 @@ class OracleSampler:
                                    kv_heads=sorted({r % wl.hkv for r in rows}))
         f = inputs.bf16_to_f64
         self.lay = A.OracleLayer(wl.batch, wl.hq, wl.hkv, wl.head_dim, wl.window, wl.n_obs,
-                                 wl.budget_frac, wl.gamma, pre["ctx_len"], rows=self.rows)
+                                 wl.budget_frac, wl.gamma, pre["ctx_len"], rows=self.rows,
+                                 fmt=wl.quant_format)
         self.lay.prefill(f(pre["k"]), f(pre["v"]), f(pre["q_obs"]))
         self.r = wl.oq_ratio if wl.oq_ratio is not None else wl.r_bar
         self.lay.initial_reassign(self.r)
@@ -186,15 +187,103 @@ class OracleSampler:
                 f"{wl.layers} layers x {wl.rows} rows")
 
 
-def cpu_baseline_line(wl, seconds):
-    smp = OracleSampler(wl)
-    per, spent = [], 0.0
-    while len(per) < wl.reassign_interval or spent < seconds:
-        per.append(smp.step())
-        spent += per[-1] * len(smp.rows)
-    step_s = statistics.mean(per) * wl.rows * wl.layers
-    return {"value": wl.batch / step_s, "unit": "tokens/s", "cores": smp.threads, "kind": "oracle",
-            "sample": smp.describe(len(per))}
+def cpu_baseline_from_state(wl, lay0, ctx_np, t_next, o_dev, seconds, decode_step_dev):
+    """The oracle on the benchmarked data: row 0 of layer 0 is read back from the device
+    after the timed passes and loaded into the oracle; one decode step is then run on
+    both (the device's step outside any timed region) and compared -- attention output
+    and scores -- and the oracle goes on alone for timed steps, first on every core,
+    then on one thread."""
+    import numpy as np
+    import torch
+    from threadpoolctl import threadpool_info, threadpool_limits
+    from mixed_precision_kv_arkv_b200 import inputs
+    from oracle import arkv as A
+
+    c, rid, D, G = lay0["cache"], 0, wl.head_dim, wl.group
+    n0 = int(ctx_np[0])
+    n16, n8 = int(c.n_bf16[rid]), int(c.n_fp8[rid])
+    f = inputs.bf16_to_f64
+    to_u16 = lambda t: t.view(torch.int16).cpu().numpy().view(np.uint16)
+    pos = np.concatenate([c.pos16[rid, :n16].cpu().numpy(), c.pos8[rid, :n8].cpu().numpy()]).astype(np.int64)
+    order = np.argsort(pos, kind="stable")
+    cat = lambda a, b: np.concatenate([a, b])[order]
+    zeros16 = np.zeros((n8, D), np.uint16)
+    row = A.Row(D=D, pos=pos[order], orig=cat(np.ones(n16, bool), np.zeros(n8, bool)),
+                kf=f(cat(to_u16(c.k16[rid, :n16]), zeros16)), vf=f(cat(to_u16(c.v16[rid, :n16]), zeros16)),
+                kc=cat(np.zeros((n16, D), np.uint8), c.k8[rid, :n8].cpu().numpy()),
+                vc=cat(np.zeros((n16, D), np.uint8), c.v8[rid, :n8].cpu().numpy()),
+                sk=cat(np.ones(n16, np.float32), c.sk[rid, :n8].cpu().numpy()),
+                sv=cat(np.ones(n16, np.float32), c.sv[rid, :n8].cpu().numpy()),
+                mu=cat(c.mu16[rid, :n16].cpu().numpy(), c.mu8[rid, :n8].cpu().numpy()),
+                m2=cat(c.m2_16[rid, :n16].cpu().numpy(), c.m2_8[rid, :n8].cpu().numpy()),
+                fmt=wl.quant_format)
+    # Welford counts after step t_next - 1: the observations the token has had
+    p_ = row.pos
+    row.cnt = np.where(p_ < n0, np.minimum(wl.n_obs, n0 - p_) + t_next, t_next - (p_ - n0)).astype(np.int64)
+
+    dec = lay0["dec"]
+    host = {k: dec[k].view(torch.int16).cpu().numpy().view(np.uint16) for k in ("q", "k_new", "v_new")}
+    n_in = host["q"].shape[0]
+
+    def oracle_step(t):
+        i = t % n_in
+        row.append(n0 + t, f(host["k_new"][i, 0, 0]), f(host["v_new"][i, 0, 0]))
+        o, _ = A.decode_row(row, f(host["q"][i, 0, :G]))
+        if (t + 1) % wl.reassign_interval == 0:
+            A.reassign_row(row, n0 + t + 1, wl.window, wl.budget_frac, lay0["r"], wl.gamma)
+        return o
+
+    # the step both sides take from the same state
+    decode_step_dev(t_next)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    o_ref = oracle_step(t_next)
+    first = time.perf_counter() - t0
+    o_gpu = o_dev[0, 0, :G].cpu().numpy().astype(np.float64)
+    o_rel = float((np.abs(o_gpu - o_ref).max(axis=-1) / np.abs(o_ref).max(axis=-1)).max())
+    check = {"o_rel": o_rel}
+    if (t_next + 1) % wl.reassign_interval != 0:   # scores of the same tokens on both sides
+        n16, n8 = int(c.n_bf16[rid]), int(c.n_fp8[rid])
+        pos2 = np.concatenate([c.pos16[rid, :n16].cpu().numpy(), c.pos8[rid, :n8].cpu().numpy()]).astype(np.int64)
+        o2 = np.argsort(pos2, kind="stable")
+        mu = np.concatenate([c.mu16[rid, :n16].cpu().numpy(), c.mu8[rid, :n8].cpu().numpy()])[o2]
+        m2 = np.concatenate([c.m2_16[rid, :n16].cpu().numpy(), c.m2_8[rid, :n8].cpu().numpy()])[o2]
+        same = np.array_equal(pos2[o2], row.pos)
+        check["positions_equal"] = bool(same)
+        if same:
+            s_ref = A.heavy_hitter_score(row.mu, row.m2, row.cnt, wl.gamma)
+            s_gpu = A.heavy_hitter_score(mu, m2, row.cnt, wl.gamma)
+            check["s_rel"] = float(np.max(np.abs(s_gpu - s_ref) / (np.abs(s_ref) + 1e-300)))
+    check["tolerance"] = {"o_rel": 2e-3, "s_rel": 1e-5}
+    check["ok"] = bool(o_rel <= 2e-3 and check.get("s_rel", 0.0) <= 1e-5 and check.get("positions_equal", True))
+
+    def timed_steps(t, budget):
+        per = [first] if t == t_next + 1 else []
+        spent = sum(per)
+        while len(per) < wl.reassign_interval or spent < budget:
+            a = time.perf_counter()
+            oracle_step(t)
+            per.append(time.perf_counter() - a)
+            spent += per[-1]
+            t += 1
+        return per, t
+
+    all_threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    per_all, t = timed_steps(t_next + 1, seconds / 2)
+    with threadpool_limits(limits=1):
+        per_one, t = timed_steps(t, seconds / 2)
+    scale = wl.rows * wl.layers                       # row-steps in one decode step of the stack
+    v_all = wl.batch / (statistics.mean(per_all) * scale)
+    v_one = wl.batch / (statistics.mean(per_one) * scale)
+    return {"value": v_all, "unit": "tokens/s", "cores": all_threads, "nproc": os.cpu_count(),
+            "kind": "oracle",
+            "single_thread": {"value": v_one, "unit": "tokens/s", "cores": 1},
+            "sample": (f"oracle on row 0 of layer 0 ({wl.name}) from the benchmarked device state after "
+                       f"{t_next} decode steps: {len(per_all)} steps on {all_threads} threads, then "
+                       f"{len(per_one)} on 1 thread, reassignments every {wl.reassign_interval}; time per "
+                       f"row-step scaled to {wl.layers} layers x {wl.rows} rows (extrapolated)"),
+            "extrapolated": True,
+            "check_on_benchmarked_state": check}
 
 
 def run_reference(args, wl, rank):
@@ -214,7 +303,9 @@ def run_reference(args, wl, rank):
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(wl),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": smp.threads,
-                             "kind": "oracle", "sample": smp.describe(len(per))},
+                             "nproc": os.cpu_count(), "kind": "oracle", "sample": smp.describe(len(per)),
+                             "extrapolated": True},
+            "extrapolated": True,
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -225,7 +316,7 @@ def config_of(wl):
             "head_dim": wl.head_dim, "n_ctx": wl.n_ctx, "n_ctx_min": wl.n_ctx_min,
             "budget_frac": wl.budget_frac, "oq_ratio": wl.oq_ratio if wl.oq_ratio is not None
             else f"per layer from prefill stats (r_bar {wl.r_bar})", "window": wl.window,
-            "gamma": wl.gamma, "reassign_interval": wl.reassign_interval,
+            "gamma": wl.gamma, "reassign_interval": wl.reassign_interval, "quant_format": wl.quant_format,
             "l2": "no flush: every step streams the whole compressed cache, far above L2"}
 
 
@@ -247,11 +338,11 @@ def run_arkv(args, wl, rank, world, local_rank):
     passes = 1 + (0 if args.no_e2e else 1) + 1          # value, e2e, kernel timing
     total_steps = W + passes * K
     ctx_np = inputs.ctx_lengths(wl, 0)
-    n_max = int(ctx_np.max()) + total_steps
+    n_max = int(ctx_np.max()) + total_steps + 1        # + the step the CPU baseline checks
     ctx = torch.from_numpy(ctx_np).to(dev)
 
     # ---------- prefill statistics of every layer, then the per-layer Original share
-    probe = make_cfg(B, Hq, Hkv, D, wl.window, wl.n_obs, wl.gamma, wl.budget_frac, 1, 1)
+    probe = make_cfg(B, Hq, Hkv, D, wl.window, wl.n_obs, wl.gamma, wl.budget_frac, 1, 1, wl.quant_format)
     ws_pre = Workspace(abi.arkv_workspace_bytes(probe, abi.ARKV_WS_PREFILL, wl.n_ctx), dev)
     stats = torch.zeros((L, 3), dtype=torch.float64, device=dev)
     mu0 = torch.zeros((wl.rows, wl.n_ctx), dtype=torch.float64, device=dev)
@@ -274,7 +365,8 @@ def run_arkv(args, wl, rank, world, local_rank):
     layers = []
     for l in range(L):
         cap_o, cap_q = abi.arkv_row_capacity(probe, n_max, float(r[l]), wl.reassign_interval)
-        cfg = make_cfg(B, Hq, Hkv, D, wl.window, wl.n_obs, wl.gamma, wl.budget_frac, cap_o, cap_q)
+        cfg = make_cfg(B, Hq, Hkv, D, wl.window, wl.n_obs, wl.gamma, wl.budget_frac, cap_o, cap_q,
+                       wl.quant_format)
         cache = LayerCache(cfg, dev)
         pre = inputs.layer_prefill_torch(wl, l, dev, seed, ctx_np)
         abi.arkv_prefill_stats(cfg, pre["q_obs"].data_ptr(), pre["k"].data_ptr(), wl.n_ctx,
@@ -283,7 +375,7 @@ def run_arkv(args, wl, rank, world, local_rank):
         abi.arkv_quantize_pack(cfg, float(r[l]), pre["k"].data_ptr(), pre["v"].data_ptr(), wl.n_ctx,
                                ctx.data_ptr(), mu0.data_ptr(), m20.data_ptr(), cache.c, None,
                                ws_pre.ptr, ws_pre.nbytes, s)
-        dec = inputs.decode_inputs_torch(wl, pre["u"], total_steps, dev, seed, l)
+        dec = inputs.decode_inputs_torch(wl, pre["u"], total_steps + 1, dev, seed, l)
         layers.append({"cfg": cfg, "cache": cache, "r": float(r[l]), "dec": dec,
                        "ws_d": Workspace(abi.arkv_workspace_bytes(cfg, abi.ARKV_WS_DECODE), dev),
                        "ws_r": Workspace(abi.arkv_workspace_bytes(cfg, abi.ARKV_WS_REASSIGN), dev)})
@@ -413,8 +505,7 @@ def run_arkv(args, wl, rank, world, local_rank):
         "hbm_gbs_step": step_bytes / (ms_value / K * 1e-3) / 1e9,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": kernel_traffic("decode_attn.cu"),
-                     "kernel": (f"arkv_decode_attn call: decode_attn_kernel<{D}> + merge_kernel<{D}> "
-                                "(timed together; algorithmic bytes are the attention's)"),
+                     "kernel": f"arkv_decode_attn call: decode_attn_kernel<{D}> (split merge fused)",
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                      else "fallback 6650 GB/s",
                      "bytes_per_launch": float(alg_bytes.mean()),
@@ -429,7 +520,8 @@ def run_arkv(args, wl, rank, world, local_rank):
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "ms_per_step": ms_e2e / K}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline_line(wl, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline_from_state(wl, layers[0], ctx_np, total_steps, o, args.cpu_seconds,
+                                                       lambda t: layer_step(0, t))
     if rank == 0:
         print(json.dumps(line), flush=True)
     del g_value, g_k

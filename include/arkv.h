@@ -69,9 +69,14 @@ typedef struct CUstream_st *arkv_stream_t;   /* same type as cudaStream_t */
 #define ARKV_TIER_QUANTIZED  1
 #define ARKV_TIER_EVICTED    2
 
+/* FP8 formats of the Quantized tier (§2.다 "low precision, e.g. FP8"; OCP FP8):
+ * codes = RNE(x / s) with saturation, s = amax / FMAX per token and head. */
+#define ARKV_FMT_E4M3  0   /* 4 exponent bits, 3 mantissa bits, FMAX = 448 (default) */
+#define ARKV_FMT_E5M2  1   /* 5 exponent bits, 2 mantissa bits, FMAX = 57344 */
+
 /* Shapes and policy of one layer.  hq % hkv == 0, hq / hkv (the query group
  * G) in 1..4, head_dim 64 or 128, window >= 1, 1 <= n_obs, budget_frac in
- * (0, 1], gamma >= 0. */
+ * (0, 1], gamma >= 0, quant_format ARKV_FMT_E4M3 or ARKV_FMT_E5M2. */
 typedef struct arkv_cfg {
     int32_t batch;
     int32_t hq;             /* query heads */
@@ -83,6 +88,7 @@ typedef struct arkv_cfg {
     float   budget_frac;    /* beta: bytes kept per row <= beta * N_t * 4D (§2.다 memory budget) */
     int32_t cap_bf16;       /* slots per row, bf16 segment */
     int32_t cap_fp8;        /* slots per row, fp8 segment */
+    int32_t quant_format;   /* ARKV_FMT_*: FP8 format of the Quantized tier */
 } arkv_cfg;
 
 /* Device buffers of one layer's packed cache (see Layout above). */
@@ -147,8 +153,8 @@ int arkv_oq_ratio(const double *stats, int32_t layers, double r_bar, float *r_ou
  * position), keeps the budget's
  * n_sel, makes the first n_o of them Original and quantizes the rest, evicts the
  * others, and writes the cache: bf16 segment = Originals + the W newest tokens,
- * fp8 segment = the Quantized tokens (codes = RNE_E4M3(x / s), s = amax / 448 in
- * float32, s = 1 if amax = 0), both in position order.  Counts follow
+ * fp8 segment = the Quantized tokens (codes = RNE_FP8(x / s), s = amax / FMAX in
+ * float32, s = 1 if amax = 0, in cfg's quant_format), both in position order.  Counts follow
  *   Rb = beta*N*4D - W*4D, n_sel = min(floor(Rb / (r*4D + (1-r)*(2D+8))), candidates),
  *   n_o = floor(r * n_sel)            (float64, operations in this order).
  *   k, v [batch][hkv][n_ctx_max][D] bf16 bits; mu0, m2_0 from arkv_prefill_stats;
@@ -166,8 +172,11 @@ int arkv_quantize_pack(const arkv_cfg *cfg, float r, const uint16_t *k, const ui
  * over the row's live tokens, with k^ = k for bf16 slots and k^ = code * scale for
  * fp8 slots (v^ likewise).  o is written in float32.  Each token's raw logits and
  * each head's softmax max and sum are left in `ws` for arkv_score_update.
- *   q [batch][hq][D], k_new, v_new [batch][hkv][D] bf16 bits; o [batch][hq][D] float.
- * A full bf16 segment sets ARKV_STATUS_BF16_FULL and drops the new token. */
+ *   q [batch][hq][D], k_new, v_new [batch][hkv][D] bf16 bits; o [batch][hq][D] float;
+ *   all four 16-byte aligned.
+ * The row's bf16 count (n_bf16) is advanced past the new token when the call
+ * completes.  A full bf16 segment sets ARKV_STATUS_BF16_FULL and drops the new
+ * token. */
 int arkv_decode_attn(const arkv_cfg *cfg, int32_t step, const uint16_t *q, const uint16_t *k_new,
                      const uint16_t *v_new, const int32_t *ctx_len, arkv_layer_cache *cache,
                      float *o, void *ws, size_t ws_bytes, arkv_stream_t stream);
@@ -200,9 +209,10 @@ int arkv_reassign(const arkv_cfg *cfg, int32_t step, float r, const int32_t *ctx
                   arkv_layer_cache *cache, uint8_t *tier_dbg, void *ws, size_t ws_bytes,
                   arkv_stream_t stream);
 
-/* The device float32 -> E4M3 conversion the quantizer uses (round to nearest
- * even, saturate to +-448), for testing: out[i] = code(x[i]), n elements. */
-int arkv_fp8_encode(const float *x, uint8_t *out, size_t n, arkv_stream_t stream);
+/* The device float32 -> FP8 conversion the quantizer uses (round to nearest
+ * even, saturate to +-FMAX) in `format` (ARKV_FMT_*), for testing:
+ * out[i] = code(x[i]), n elements. */
+int arkv_fp8_encode(int32_t format, const float *x, uint8_t *out, size_t n, arkv_stream_t stream);
 
 /* Allocation-free tier reassignment.  The paper has no counterpart: this is an
  * interface for callers that cannot allocate device memory when they reassign --

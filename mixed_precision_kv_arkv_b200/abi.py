@@ -16,6 +16,8 @@ ARKV_OK, ARKV_EINVAL, ARKV_ECAPACITY, ARKV_ECUDA = 0, -1, -2, -3
 ARKV_STATUS_BF16_FULL, ARKV_STATUS_FP8_FULL = 1, 2
 ARKV_TIER_ORIGINAL, ARKV_TIER_QUANTIZED, ARKV_TIER_EVICTED = 0, 1, 2
 ARKV_WS_DECODE, ARKV_WS_REASSIGN, ARKV_WS_PREFILL = 0, 1, 2
+ARKV_FMT_E4M3, ARKV_FMT_E5M2 = 0, 1
+FORMATS = {"e4m3": ARKV_FMT_E4M3, "e5m2": ARKV_FMT_E5M2}
 ARKV_NOALLOC_SCRATCH_BYTES = 24 << 20
 
 
@@ -23,7 +25,8 @@ class arkv_cfg(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("hq", ctypes.c_int32), ("hkv", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("window", ctypes.c_int32), ("n_obs", ctypes.c_int32),
                 ("gamma", ctypes.c_float), ("budget_frac", ctypes.c_float),
-                ("cap_bf16", ctypes.c_int32), ("cap_fp8", ctypes.c_int32)]
+                ("cap_bf16", ctypes.c_int32), ("cap_fp8", ctypes.c_int32),
+                ("quant_format", ctypes.c_int32)]
 
 
 class arkv_layer_cache(ctypes.Structure):
@@ -52,7 +55,7 @@ _SIG = {
     "arkv_score_update": (ctypes.c_int, [_P, ctypes.c_int32, _P, _P, _P, ctypes.c_size_t, _P]),
     "arkv_reassign": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_float, _P, _P, _P, _P,
                                      ctypes.c_size_t, _P]),
-    "arkv_fp8_encode": (ctypes.c_int, [_P, _P, ctypes.c_size_t, _P]),
+    "arkv_fp8_encode": (ctypes.c_int, [ctypes.c_int32, _P, _P, ctypes.c_size_t, _P]),
     "arkv_reassign_noalloc": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_float, _P, _P, _P, _P]),
     "arkv_last_error_string": (ctypes.c_char_p, []),
 }
@@ -142,6 +145,6 @@ def arkv_reassign_noalloc(cfg, step, r, ctx_len, cache, tier_dbg, stream, check=
     return _check("arkv_reassign_noalloc", rc) if check else rc
 
 
-def arkv_fp8_encode(x, out, n, stream, check=True) -> int:
-    rc = lib().arkv_fp8_encode(x, out, n, stream)
+def arkv_fp8_encode(fmt, x, out, n, stream, check=True) -> int:
+    rc = lib().arkv_fp8_encode(fmt, x, out, n, stream)
     return _check("arkv_fp8_encode", rc) if check else rc

@@ -11,9 +11,10 @@ import torch
 from . import abi
 
 
-def make_cfg(batch, hq, hkv, head_dim, window, n_obs, gamma, budget_frac, cap_bf16, cap_fp8):
+def make_cfg(batch, hq, hkv, head_dim, window, n_obs, gamma, budget_frac, cap_bf16, cap_fp8,
+             quant_format="e4m3"):
     return abi.arkv_cfg(batch, hq, hkv, head_dim, window, n_obs, float(gamma), float(budget_frac),
-                        cap_bf16, cap_fp8)
+                        cap_bf16, cap_fp8, abi.FORMATS[quant_format])
 
 
 class LayerCache:

@@ -37,6 +37,8 @@ int check_cfg(const arkv_cfg* c) {
     if (!(c->budget_frac > 0.f && c->budget_frac <= 1.f))
         return fail(ARKV_EINVAL, "%s: budget_frac must be in (0, 1]", "cfg");
     if (c->cap_bf16 < 1 || c->cap_fp8 < 1) return fail(ARKV_EINVAL, "%s: capacities must be >= 1", "cfg");
+    if (c->quant_format != ARKV_FMT_E4M3 && c->quant_format != ARKV_FMT_E5M2)
+        return fail(ARKV_EINVAL, "%s: quant_format must be ARKV_FMT_E4M3 or ARKV_FMT_E5M2", "cfg");
     return ARKV_OK;
 }
 
@@ -45,6 +47,7 @@ arkv::LayerDims dims(const arkv_cfg* c) {
     d.batch = c->batch; d.hq = c->hq; d.hkv = c->hkv; d.G = c->hq / c->hkv; d.D = c->head_dim;
     d.W = c->window; d.n_obs = c->n_obs; d.gamma = c->gamma; d.beta = c->budget_frac;
     d.cap_o = c->cap_bf16; d.cap_q = c->cap_fp8; d.R = c->batch * c->hkv;
+    d.fmt = c->quant_format;
     return d;
 }
 
@@ -78,22 +81,6 @@ int check_ws(const void* ws, size_t have, size_t need) {
         if (_rc != ARKV_OK) return _rc; \
     } while (0)
 
-struct PrefillWs {
-    size_t sumx, qstat, keys, idx, total;
-};
-
-PrefillWs prefill_ws(const arkv::LayerDims& d, int n_stride) {
-    auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    PrefillWs w{};
-    size_t off = 0;
-    w.sumx = off;  off = al(off + sizeof(double) * (size_t)d.R * n_stride * 2);
-    w.qstat = off; off = al(off + sizeof(double) * (size_t)d.batch * d.hq * d.n_obs * 3);
-    w.keys = off;  off = al(off + sizeof(uint64_t) * (size_t)d.R * n_stride);
-    w.idx = off;   off = al(off + sizeof(int32_t) * (size_t)d.R * n_stride);
-    w.total = off;
-    return w;
-}
-
 }  // namespace
 
 void arkv::set_last_error(const char* msg) { snprintf(g_err, sizeof g_err, "%s", msg); }
@@ -108,7 +95,7 @@ size_t arkv_workspace_bytes(const arkv_cfg* cfg, int which, int32_t n_ctx_max) {
     switch (which) {
         case ARKV_WS_DECODE: return arkv::decode_ws_layout(d).total;
         case ARKV_WS_REASSIGN: return arkv::reassign_ws_bytes(d);
-        case ARKV_WS_PREFILL: return n_ctx_max > 0 ? prefill_ws(d, n_ctx_max).total : 0;
+        case ARKV_WS_PREFILL: return n_ctx_max > 0 ? arkv::prefill_ws_layout(d, n_ctx_max).total : 0;
         default: return 0;
     }
 }
@@ -154,14 +141,15 @@ int arkv_prefill_stats(const arkv_cfg* cfg, const uint16_t* q_obs, const uint16_
         return fail(ARKV_EINVAL, "%s: q_obs and k must be 16-byte aligned", "arkv_prefill_stats");
     if (n_ctx_max < cfg->n_obs) return fail(ARKV_EINVAL, "%s: n_ctx_max < n_obs", "arkv_prefill_stats");
     const arkv::LayerDims d = dims(cfg);
-    const PrefillWs w = prefill_ws(d, n_ctx_max);
+    const arkv::PrefillWs w = arkv::prefill_ws_layout(d, n_ctx_max);
     ARKV_TRY(check_ws(ws, ws_bytes, w.total));
     arkv::PrefillParams p{};
     p.d = d; p.q_obs = q_obs; p.k = k; p.n_stride = n_ctx_max; p.ctx_len = ctx_len;
     p.stats_out = stats_out;
     p.query_stats = query_stats ? query_stats : (double*)((char*)ws + w.qstat);
     p.mu0 = mu0; p.m2_0 = m2_0;
-    p.sumx = (double*)((char*)ws + w.sumx);
+    p.part = (double*)((char*)ws + w.part);
+    p.qml = (double*)((char*)ws + w.qml);
     const cudaError_t e = arkv::launch_prefill_stats(p, (cudaStream_t)stream);
     return e == cudaSuccess ? ARKV_OK : cuda_fail(e, "arkv_prefill_stats");
 }
@@ -180,7 +168,7 @@ int arkv_quantize_pack(const arkv_cfg* cfg, float r, const uint16_t* k, const ui
     if (cfg->cap_bf16 < n_o + cfg->window || cfg->cap_fp8 < n_sel - n_o)
         return fail(ARKV_ECAPACITY, "%s: capacities below the kept counts at n_ctx_max", "arkv_quantize_pack");
     const arkv::LayerDims d = dims(cfg);
-    const PrefillWs w = prefill_ws(d, n_ctx_max);
+    const arkv::PrefillWs w = arkv::prefill_ws_layout(d, n_ctx_max);
     ARKV_TRY(check_ws(ws, ws_bytes, w.total));
     arkv::PackParams p{};
     p.d = d; p.r = r; p.k = k; p.v = v; p.n_stride = n_ctx_max; p.ctx_len = ctx_len; p.mu0 = mu0; p.m2_0 = m2_0;
@@ -197,8 +185,8 @@ int arkv_decode_attn(const arkv_cfg* cfg, int32_t step, const uint16_t* q, const
     ARKV_TRY(check_cfg(cfg));
     ARKV_TRY(check_cache(cache));
     if (!q || !k_new || !v_new || !ctx_len || !o) return fail(ARKV_EINVAL, "%s: null argument", "arkv_decode_attn");
-    if (!aligned(q, 16) || !aligned(k_new, 16) || !aligned(v_new, 16))
-        return fail(ARKV_EINVAL, "%s: q, k_new, v_new must be 16-byte aligned", "arkv_decode_attn");
+    if (!aligned(q, 16) || !aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(o, 16))
+        return fail(ARKV_EINVAL, "%s: q, k_new, v_new and o must be 16-byte aligned", "arkv_decode_attn");
     if (step < 0) return fail(ARKV_EINVAL, "%s: step < 0", "arkv_decode_attn");
     const arkv::LayerDims d = dims(cfg);
     const arkv::DecodeWs w = arkv::decode_ws_layout(d);
@@ -212,8 +200,8 @@ int arkv_decode_attn(const arkv_cfg* cfg, int32_t step, const uint16_t* q, const
     p.part_ml = (float2*)(base + w.part_ml);
     p.ml = (float2*)(base + w.ml);
     p.counter = (unsigned*)(base + w.counter);
-    p.nsplit_o = w.nsplit_o;
-    p.nsplit_q = w.nsplit_q;
+    p.lstride_o = w.lstride_o;
+    p.lstride_q = w.lstride_q;
     p.inv_sqrt_d = 1.0 / sqrt((double)d.D);
     const cudaError_t e = arkv::launch_decode_attn(p, (cudaStream_t)stream);   // also encodes the tensor maps
     return e == cudaSuccess ? ARKV_OK : cuda_fail(e, "arkv_decode_attn");
@@ -234,6 +222,8 @@ int arkv_score_update(const arkv_cfg* cfg, int32_t step, const int32_t* ctx_len,
     p.logit16 = (const float*)(base + w.logit16);
     p.logit8 = (const float*)(base + w.logit8);
     p.ml = (const float2*)(base + w.ml);
+    p.lstride_o = w.lstride_o;
+    p.lstride_q = w.lstride_q;
     p.inv_sqrt_d = 1.0 / sqrt((double)d.D);
     const cudaError_t e = arkv::launch_score_update(p, (cudaStream_t)stream);
     return e == cudaSuccess ? ARKV_OK : cuda_fail(e, "arkv_score_update");
@@ -259,9 +249,11 @@ int arkv_reassign(const arkv_cfg* cfg, int32_t step, float r, const int32_t* ctx
     return e == cudaSuccess ? ARKV_OK : cuda_fail(e, "arkv_reassign");
 }
 
-int arkv_fp8_encode(const float* x, uint8_t* out, size_t n, arkv_stream_t stream) {
+int arkv_fp8_encode(int32_t format, const float* x, uint8_t* out, size_t n, arkv_stream_t stream) {
+    if (format != ARKV_FMT_E4M3 && format != ARKV_FMT_E5M2)
+        return fail(ARKV_EINVAL, "%s: unknown format", "arkv_fp8_encode");
     if (n > 0 && (!x || !out)) return fail(ARKV_EINVAL, "%s: null argument", "arkv_fp8_encode");
-    const cudaError_t e = arkv::launch_fp8_encode(x, out, n, (cudaStream_t)stream);
+    const cudaError_t e = arkv::launch_fp8_encode(format, x, out, n, (cudaStream_t)stream);
     return e == cudaSuccess ? ARKV_OK : cuda_fail(e, "arkv_fp8_encode");
 }
 

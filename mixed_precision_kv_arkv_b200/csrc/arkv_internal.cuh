@@ -12,9 +12,6 @@
 namespace arkv {
 
 constexpr int kGP = 4;                 // query-group width the kernels are laid out for
-constexpr int kAttnThreads = 128;      // decode attention CTA: 4 warps
-constexpr int kSplitBf16 = 256;        // bf16 tokens per decode CTA
-constexpr int kSplitFp8 = 512;         // fp8 tokens per decode CTA
 constexpr int kRowThreads = 1024;      // one CTA per row for selection / compaction
 
 // ------------------------------------------------------------------ numerics
@@ -88,21 +85,24 @@ __host__ __device__ inline void budget_counts(float beta, int n_t, float r, int 
 }
 
 // Quantize one token-head vector held by a warp (EPL elements per lane, lane l
-// holds elements [l*EPL, (l+1)*EPL)): s = amax / 448 (1 if amax == 0), codes =
-// RNE_E4M3(x / s) with saturation.  Writes EPL codes per lane and returns s.
-template <int EPL>
+// holds elements [l*EPL, (l+1)*EPL)) to FP8 in format FMT (ARKV_FMT_*):
+// s = amax / FMAX (1 if amax == 0), codes = RNE_FP8(x / s) with saturation.
+// Writes EPL codes per lane and returns s.
+template <int EPL, int FMT>
 __device__ __forceinline__ float quantize_warp(const float (&x)[EPL], uint8_t* codes_out) {
+    constexpr float kFmax = FMT == ARKV_FMT_E5M2 ? 57344.0f : 448.0f;
+    constexpr __nv_fp8_interpretation_t kInterp = FMT == ARKV_FMT_E5M2 ? __NV_E5M2 : __NV_E4M3;
     float amax = 0.f;
 #pragma unroll
     for (int e = 0; e < EPL; ++e) amax = fmaxf(amax, fabsf(x[e]));
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
-    const float s = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
+    const float s = amax == 0.f ? 1.0f : __fdiv_rn(amax, kFmax);
     uint8_t c[EPL];
 #pragma unroll
     for (int e = 0; e < EPL; e += 2) {
         float2 y = make_float2(__fdiv_rn(x[e], s), __fdiv_rn(x[e + 1], s));
-        __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);
+        __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, kInterp);
         c[e] = (uint8_t)(p & 0xff);
         c[e + 1] = (uint8_t)(p >> 8);
     }
@@ -117,6 +117,7 @@ struct LayerDims {
     float gamma, beta;
     int cap_o, cap_q;
     int R;
+    int fmt;   // ARKV_FMT_* of the Quantized tier
 };
 
 struct AttnParams {
@@ -130,13 +131,13 @@ struct AttnParams {
     const int32_t* ctx_len;
     arkv_layer_cache c;
     float* o;
-    float* logit16;     // [R][cap_o][4]
-    float* logit8;      // [R][cap_q][4]
-    float* part_o;      // [R][nsplit][4][D]
-    float2* part_ml;    // [R][nsplit][4]
+    float* logit16;     // [R][4][lstride_o] raw logits of every head, by slot
+    float* logit8;      // [R][4][lstride_q]
+    float* part_o;      // [parts][4][D]  one partial per CTA
+    float2* part_ml;    // [parts][4]
     float2* ml;         // [R][4]  final (max, sum) per head
-    unsigned* counter;  // [R]
-    int nsplit_o, nsplit_q;
+    unsigned* counter;  // [R]  the rows' tickets (zero between calls)
+    int lstride_o, lstride_q;
     double inv_sqrt_d;
 };
 
@@ -148,6 +149,7 @@ struct ScoreParams {
     const float* logit16;
     const float* logit8;
     const float2* ml;
+    int lstride_o, lstride_q;
     double inv_sqrt_d;
 };
 
@@ -155,7 +157,8 @@ struct ScoreParams {
 // arkv_score_update.
 struct DecodeWs {
     size_t logit16, logit8, part_o, part_ml, ml, counter, total;
-    int nsplit_o, nsplit_q;
+    int parts;                       // partial slots: the largest grid of one call
+    int lstride_o, lstride_q;
 };
 DecodeWs decode_ws_layout(const LayerDims& d);
 
@@ -198,17 +201,21 @@ struct PrefillParams {
     int n_stride;
     const int32_t* ctx_len;
     double* stats_out;
-    double* query_stats;    // [B][Hq][n_obs][3] or null
+    double* query_stats;    // [B][Hq][n_obs][3]
     double* mu0;
     double* m2_0;
-    double* qml;            // ws [B][Hq][n_obs][2]   (max, sum) per query
-    double* qstat;          // ws [B][Hq][n_obs][3]
-    double* sumx;           // ws [R][n_stride][2]    (sum x, sum x^2) per key
+    double* part;           // ws [R][n_obs][4][key ranges][6] partial sums of the sweep
+    double* qml;            // ws [R][n_obs][4][2] final (max, sum) per query
 };
-size_t prefill_ws_bytes(const LayerDims& d, int n_stride);
+// Prefill workspace layout (byte offsets), shared by arkv_prefill_stats and
+// arkv_quantize_pack (keys, idx).
+struct PrefillWs {
+    size_t part, qml, qstat, keys, idx, total;
+};
+PrefillWs prefill_ws_layout(const LayerDims& d, int n_stride);
 cudaError_t launch_prefill_stats(const PrefillParams& p, cudaStream_t s);
 
-cudaError_t launch_fp8_encode(const float* x, uint8_t* out, size_t n, cudaStream_t s);
+cudaError_t launch_fp8_encode(int fmt, const float* x, uint8_t* out, size_t n, cudaStream_t s);
 
 // Replace the calling thread's last-error message (see arkv_last_error_string).
 void set_last_error(const char* msg);

@@ -2,32 +2,42 @@
 // are dequantized right before attention and attended together with the
 // originals) and the score observation that feeds §2.나.
 //
-// One CTA per split of one row: kSplitBf16 consecutive bf16 slots or kSplitFp8
-// consecutive fp8 slots, 4 warps.  Each warp streams every fourth 16-token tile
-// of the split through its own ring of kStages shared-memory stages, filled by
-// TMA tensor loads (16 rows x 128 bytes per box, 128-byte swizzle) completing on
-// per-stage mbarriers (waits are bounded).
+// One wave of CTAs (as many as the GPU holds at once) shares the rows in
+// proportion to their lengths; each CTA takes an equal share of its row, counted
+// in 16-token tiles (a bf16 tile weighs two FP8 tiles, its bytes), bf16 tiles first
+// and FP8 tiles after.  Its 4 warps take the tiles round robin, each through its
+// own ring of 4 shared-memory slots (a bf16 tile takes two, K then V; an FP8 tile
+// one) filled by TMA tensor loads (16 rows per box, 128-byte swizzle; 64-byte for
+// FP8 rows of 64 bytes) completing on per-slot mbarriers (waits are bounded).
 //
-// Per tile the query group's heads (G <= 4) meet the tile on the tensor cores,
-// warp-level m16n8k16:
-//   S^T[16 tok][8] = K[16 tok][D] * Q^T[D][8]        (heads 0..3, columns 4..7 zero)
-// with one accumulator per 16-wide k block (summed afterwards in float32), and
-//   O^T[D][8] += V^T[D][16 tok] * [P_hi | P_lo][16 tok][8]
-// where the high and low halves of P fill the mma's 8 columns (heads 0..3 high,
-// 4..7 low), so that one mma keeps ~16 significant bits of every probability.
-// bf16 tiles feed the mma directly (ldmatrix, ldmatrix.trans).  FP8 tiles are
-// converted to f16 (exact for E4M3): K fragments from 4-byte loads, V^T fragments
-// from the 8-bit transposing ldmatrix (m16n16.trans.b8: lane (g, t) receives
-// tokens 4t..4t+3 at dims g and g+8, so the k positions 2t, 2t+1 | 2t+8, 2t+9
-// carry tokens 4t, 4t+1 | 4t+2, 4t+3 and P's rows are permuted to match).  The
-// per-token K scale multiplies the finished logit; the V scale is folded into P
-// relative to the largest V scale the warp will meet, and the constant comes
-// back out of the warp's partial.  The softmax runs in float32 registers with a
-// reference maximum that moves only when a logit exceeds it by 2^8 (so most
-// tiles need no cross-lane reduction); raw logits go to the workspace for the
-// score update.  The CTA combines its warps
-// into one (max, sum, unnormalised o) partial per split; merge_kernel combines a
-// row's splits and writes o.
+// Tile math on the warp-level tensor cores (m16n8k16).  QK^T with the queries as
+// the M rows: rows 0..3 and 4..7 both hold the group's heads (zero past G), rows
+// 8..15 are zero, so lane (g, t) finds the logits of head g & 3 for tokens 2t,
+// 2t+1 (n-tile 0) and 8+2t, 9+2t (n-tile 1) -- exactly the entries of the B
+// fragment of [P_hi | P_lo] that it supplies for column g of
+//   O^T[D x 8] += V^T[D x 16 tok] * [P_hi | P_lo][16 tok x 8]
+// (columns 0..3: the 16-bit high part of each head's probabilities, 4..7 the low
+// part p - hi, so one mma carries ~16 significant bits of every probability).  P
+// never leaves the registers; hi and lo meet once at the end (lanes t, t ^ 2).
+//   bf16 tiles: K fragments by ldmatrix, V^T fragments by ldmatrix.trans.
+//   FP8 tiles: codes are converted to f16 in registers (exact; E5M2 is the high
+//   byte of an f16, E4M3 goes through the hardware conversion).  K: each 4-byte
+//   word a lane reads (dims 4t..4t+3 of a 16-dim chunk) is its B fragment for that
+//   k block, and the query is loaded with the same dimension order; V: the 8-bit
+//   transposing ldmatrix gives lane (g, t) the four rows its address lanes
+//   4t..4t+3 supplied, and the rows are supplied in the token order 0,1,8,9,
+//   2,3,10,11, ... so that they are tokens 2t, 2t+1, 8+2t, 9+2t -- the k positions
+//   of the bf16 path.  The per-token K scale multiplies the finished logit; the V
+//   scale is folded into P, and every tile's P is multiplied by 64 / (the largest V
+//   scale of the warp's FP8 tiles), which keeps p * sv inside f16 and comes back
+//   out of the partial.
+// Softmax in float32 with a reference maximum that moves only when a logit
+// exceeds it by 2^8 (so most tiles need no reduction, which is two shuffles over
+// the 4 lanes of a row when it happens).  Raw logits go to the workspace for the
+// score update.  The CTA combines its warps into one (max, sum, unnormalised o)
+// partial; the last CTA of a row to finish (a ticket in the workspace) merges the
+// row's partials into o and each head's final (max, sum), and advances the row's
+// bf16 count past the appended token.
 #include <math.h>
 #include <mutex>
 
@@ -42,38 +52,43 @@ namespace {
 constexpr float kNegInf = -INFINITY;
 constexpr unsigned kFull = 0xffffffffu;
 
-#ifndef ARKV_STAGES
-#define ARKV_STAGES 2
+#ifndef ARKV_MIN_CTAS
+#define ARKV_MIN_CTAS 3
 #endif
-constexpr int kStages = ARKV_STAGES;     // tiles in flight per warp
+#ifndef ARKV_QK_CHAINS
+#define ARKV_QK_CHAINS 2
+#endif
+constexpr int kQkChains = ARKV_QK_CHAINS;   // independent QK^T accumulator chains per n-tile
 constexpr int kWarps = 4;
-constexpr int kSpinLimit = 1 << 20;      // bounded mbarrier waits (~1 s worst case)
+constexpr int kSlots = 4;                  // ring slots per warp: a bf16 tile takes 2, an FP8 tile 1
+constexpr int kSpinLimit = 1 << 20;        // bounded mbarrier waits (~1 s worst case)
+constexpr int kMaxGrid = 2048;             // CTAs of one call at most (partial slots in the workspace)
 
 // ------------------------------------------------------------------ shared-memory layout
 template <int D>
 struct Smem {
-    static constexpr int kTileBytes = 16 * D * 2;                       // 16 rows of bf16
-    static constexpr int kStage = 2 * kTileBytes;                       // K tile then V tile
-    static constexpr int kRing = kWarps * kStages * kStage;
-    static constexpr int kBars = kRing;                                 // uint64 [4][kStages]
-    static constexpr int kP = kBars + kWarps * kStages * 8;             // float [4][16][8]
-    static constexpr int kM = kP + kWarps * 16 * 8 * 4;                 // float [4][4]
+    static constexpr int kSlot = 16 * D * 2;                            // 16 rows of bf16: one K or V tile
+    static constexpr int kRing = kWarps * kSlots * kSlot;
+    static constexpr int kBars = kRing;                                 // uint64 [4][kSlots]
+    static constexpr int kM = kBars + kWarps * kSlots * 8;              // float [4][4]
     static constexpr int kL = kM + 16 * 4;                              // float [4][4]
     static constexpr int kRed = kL + 16 * 4;                            // float [4][4]
     static constexpr int kMax = kRed + 16 * 4;                          // float [4]
     static constexpr int kAbort = kMax + 16;                            // int: a wait gave up
-    static constexpr int kBytes = kAbort + 16 + 1024;                   // + alignment slack
+    static constexpr int kShare = kAbort + 16;                          // int [4]: row, index, count, base
+    static constexpr int kBytes = kShare + 16 + 1024;                   // + alignment slack
     static constexpr int kO = 0;                                        // float [4][4][D], in the idle ring
     static_assert(4 * 4 * D * 4 <= kRing, "the epilogue buffer must fit in the ring");
 };
 
-// Byte offset of (row, byte) in a 16-row tile of `rowb`-byte rows written by a TMA
-// load with the matching swizzle (128-byte rows: 16-byte chunks XOR row % 8;
-// 64-byte rows: XOR (row / 2) % 4).  Tiles sit at 1024-byte aligned addresses.
+// Byte offset of 16-byte chunk `chunk` of row `row` in a tile of `ROWB`-byte rows
+// written by a TMA load with the matching swizzle (128-byte rows: chunk XOR
+// row % 8; 64-byte rows: chunk XOR (row / 2) % 4).  Tiles sit at 1024-byte
+// aligned addresses.
 template <int ROWB>
-__device__ __forceinline__ int swz(int row, int byte) {
-    if constexpr (ROWB == 128) return row * 128 + (byte ^ ((row & 7) << 4));
-    else return row * 64 + (byte ^ (((row >> 1) & 3) << 4));
+__device__ __forceinline__ uint32_t swz_chunk(int row, int chunk) {
+    if constexpr (ROWB == 128) return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+    else return (uint32_t)(row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4));
 }
 
 // ------------------------------------------------------------------ PTX helpers
@@ -81,75 +96,77 @@ __device__ __forceinline__ uint32_t smem_u32(const void* ptr) {
     return (uint32_t)__cvta_generic_to_shared(ptr);
 }
 
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
 // 2-D tiled TMA load (no multicast) of the box at (x, y) completing on `bar`.
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-        "[%4];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        "[%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
         : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(bar), "r"(parity)
         : "memory");
     return ok != 0;
 }
 
 // Waits for a phase of `bar` at most kSpinLimit polls; false if it gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     for (int i = 0; i < kSpinLimit; ++i)
         if (mbar_try_wait(bar, parity)) return true;
     return false;
 }
 
+// d += a * b on m16n8k16 (f16 or bf16 operands, float32 accumulate).
 template <bool F16>
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
     if constexpr (F16)
         asm volatile(
             "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
             "{%0,%1,%2,%3};"
             : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
     else
         asm volatile(
             "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
             "{%0,%1,%2,%3};"
             : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const void* ptr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(smem_u32(ptr)));
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* ptr) {
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(smem_u32(ptr)));
+                 : "r"(addr));
 }
 
-// 16 x 16 bytes, transposed: lane (g, t) receives rows 4t..4t+3 (of the row
-// addresses lanes 0..15 supply, in that order) at columns g (r0) and g + 8 (r1).
-__device__ __forceinline__ void ldsm_b8_trans(uint32_t& r0, uint32_t& r1, const void* ptr) {
-    asm volatile("ldmatrix.sync.aligned.m16n16.x1.trans.shared.b8 {%0,%1}, [%2];"
-                 : "=r"(r0), "=r"(r1)
-                 : "r"(smem_u32(ptr)));
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// Two 16 x 16-byte matrices, transposed (rows from lanes 0..15, then 16..31): lane
+// (g, t) receives, of each matrix, the rows its lanes 4t..4t+3 supplied at byte
+// column g (r[0], r[2]) and g + 8 (r[1], r[3]).
+__device__ __forceinline__ void ldsm_b8_x2_trans(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m16n16.x2.trans.shared.b8 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -162,354 +179,453 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Two E4M3 codes (low byte first) -> f16x2, exact.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair) {
-    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(pair & 0xffffu), __NV_E4M3);
-    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+// Four FP8 codes (low byte first) -> two f16x2 words (codes 0,1 and 2,3), exact.
+// E4M3: the hardware conversion.  E5M2 is the upper byte of an f16 with the same
+// value, so the codes only move into place.
+template <int FMT>
+__device__ __forceinline__ void fp8x4_to_f16(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    if constexpr (FMT == ARKV_FMT_E5M2) {
+        lo = __byte_perm(w, 0u, 0x1404);   // bytes: 0, code 0, 0, code 1
+        hi = __byte_perm(w, 0u, 0x3424);   // bytes: 0, code 2, 0, code 3
+    } else {
+        asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+            "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n}"
+            : "=r"(lo), "=r"(hi)
+            : "r"(w));
+    }
 }
 
-// ------------------------------------------------------------------ one tile
-// Fragment conventions of m16n8k16: g = lane / 4, t = lane % 4.  ks: the stage
-// (K tile, V tile at +VOFF); tokens t0 .. t0+15 of a segment ending at seg_end.
-// sk*/sv*: the FP8 scales of this lane's tokens t0+g, t0+g+8 (1 for bf16);
-// vnorm: the warp's V-scale normaliser (FP8): 64 / the largest V scale of the warp's tiles.
-template <int D, bool FP8>
-__device__ __forceinline__ void attend_tile(const char* ks, int t0, int seg_end, int G, float c2, float skA,
-                                            float skB, float svA, float svB, float vnorm, float* logit_row,
-                                            const uint32_t (&qb)[D / 16][2], float (&m_run)[2],
-                                            float (&l_run)[2], float (&oacc)[D / 16][4], float (*sm_p)[8]) {
-    constexpr int KB = D / 16;                       // k blocks (QK^T) and m tiles (PV)
-    constexpr int ROWB = FP8 ? D : 128;              // bytes per row of one TMA box
-    constexpr int VOFF = Smem<D>::kTileBytes;
-    const int lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const char* vs = ks + VOFF;
-    const int tokA = t0 + g, tokB = t0 + g + 8;          // this lane's two tokens (QK^T rows)
-    const bool okA = tokA < seg_end, okB = tokB < seg_end;
-    const bool h0ok = 2 * t < G, h1ok = 2 * t + 1 < G;   // heads of this lane's logits
+// 2^x, the special-function unit's approximation (relative error a few 2^-23).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
-    // ---- S^T = K Q^T, one accumulator per k block, summed in float32
-    float sacc[KB][4];
+// ------------------------------------------------------------------ per-lane addresses
+// Shared-memory byte offsets (from a tile's first ring slot) of the fragment loads
+// of one lane; index j = 0..3 selects a 32-byte column pair (two 16-byte chunks) of
+// the row.  A bf16 tile holds K in its first slot and V in the next; an FP8 tile
+// holds K and V (16 x D bytes each) in one slot.  Fragment conventions of
+// m16n8k16: lane = 4 g + t.
+template <int D, bool FP8>
+struct LaneOffsets {
+    uint32_t k[4], v[4];
+    __device__ __forceinline__ LaneOffsets() {
+        const int lane = threadIdx.x & 31, m = lane >> 3;
+        constexpr int VOFF = FP8 ? 16 * D : Smem<D>::kSlot;
+        if constexpr (!FP8) {
+            // K, ldmatrix.x4: matrix m = (tokens 8 (m >> 1) .., chunk 2j + (m & 1)) -> the
+            // B fragments (b0, b1) of n-tiles 0 and 1 for k block j (16 dims = 2 chunks).
+            // V, ldmatrix.x4.trans, the same matrices -> the A fragment (a0, a1, a2, a3)
+            // of V^T for the 16 dims of block j
+            const int tk = (lane & 7) + 8 * (m >> 1);
 #pragma unroll
-    for (int kk = 0; kk < KB; ++kk) {
-        uint32_t a[4];
-        if constexpr (FP8) {
-            // k positions (2t, 2t+1 | 2t+8, 2t+9) <- dims 16 kk + 4t + (0, 1 | 2, 3)
-            const uint32_t wA = *reinterpret_cast<const uint32_t*>(ks + swz<ROWB>(g, 16 * kk + 4 * t));
-            const uint32_t wB = *reinterpret_cast<const uint32_t*>(ks + swz<ROWB>(g + 8, 16 * kk + 4 * t));
-            a[0] = e4m3x2_to_f16x2(wA);
-            a[2] = e4m3x2_to_f16x2(wA >> 16);
-            a[1] = e4m3x2_to_f16x2(wB);
-            a[3] = e4m3x2_to_f16x2(wB >> 16);
+            for (int j = 0; j < 4; ++j) {
+                k[j] = swz_chunk<128>(tk, (2 * j + (m & 1)) & 7);
+                v[j] = VOFF + k[j];
+            }
         } else {
-            // ldmatrix x4: lane l supplies row (l & 7) + 8 ((l >> 3) & 1), dims 16 kk + 8 (l >> 4)
-            const int r = (lane & 7) + 8 * ((lane >> 3) & 1);
-            const int byte = 32 * kk + 16 * (lane >> 4);
-            ldsm_x4(a, ks + (byte >> 7) * 2048 + swz<128>(r, byte & 127));
-        }
-        sacc[kk][0] = sacc[kk][1] = sacc[kk][2] = sacc[kk][3] = 0.f;
-        mma16816<FP8>(sacc[kk], a, qb[kk][0], qb[kk][1]);
-    }
+            constexpr int ROWB = D;   // one byte per dimension
+            // K, ldmatrix.x4 of 8 rows x 16 bytes: lane (g, t) receives bytes 4t..4t+3
+            // of token g (+8 for matrices 2, 3) in chunk 2j + (m & 1)
+            const int tk = (lane & 7) + 8 * (m >> 1);
+            // V, ldmatrix.m16n16.x2.trans.b8: lanes 0..15 supply the rows of matrix 0
+            // (chunk 2j), lanes 16..31 those of matrix 1 (chunk 2j + 1), in the token
+            // order 0,1,8,9,2,3,10,11,4,5,12,13,6,7,14,15
+            const int i = lane & 15;
+            const int tv = (i >> 2) * 2 + (i & 1) + 8 * ((i >> 1) & 1);
 #pragma unroll
-    for (int w = KB / 2; w >= 1; w >>= 1)
-#pragma unroll
-        for (int kk = 0; kk < w; ++kk)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sacc[kk][e] += sacc[kk + w][e];
-    // this lane: tokens A = g, B = g + 8; heads 2t, 2t+1 (t >= 2: zero columns)
-    float s[4] = {sacc[0][0], sacc[0][1], sacc[0][2], sacc[0][3]};
-    if constexpr (FP8) {
-        s[0] *= skA; s[1] *= skA; s[2] *= skB; s[3] *= skB;
-    }
-    if (t < 2) {
-        if (okA) *reinterpret_cast<float2*>(logit_row + (size_t)tokA * 4 + 2 * t) = make_float2(s[0], s[1]);
-        if (okB) *reinterpret_cast<float2*>(logit_row + (size_t)tokB * 4 + 2 * t) = make_float2(s[2], s[3]);
-    }
-    const bool v0 = okA && h0ok, v1 = okA && h1ok, v2 = okB && h0ok, v3 = okB && h1ok;
-    // online softmax for heads 2t, 2t+1 (uniform over the lanes sharing t), with a
-    // lazy reference: it moves only when a logit exceeds it by more than 8 in log2
-    // units, so probabilities stay below 2^8 and most tiles skip the reductions
-    const bool need = (v0 && (s[0] - m_run[0]) * c2 > 8.f) || (v1 && (s[1] - m_run[1]) * c2 > 8.f) ||
-                      (v2 && (s[2] - m_run[0]) * c2 > 8.f) || (v3 && (s[3] - m_run[1]) * c2 > 8.f);
-    float al0 = 1.f, al1 = 1.f;
-    if (__any_sync(kFull, need)) {
-        float mx0 = fmaxf(v0 ? s[0] : kNegInf, v2 ? s[2] : kNegInf);
-        float mx1 = fmaxf(v1 ? s[1] : kNegInf, v3 ? s[3] : kNegInf);
-#pragma unroll
-        for (int m = 4; m < 32; m <<= 1) {
-            mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, m));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, m));
-        }
-        const float n0 = fmaxf(m_run[0], mx0), n1 = fmaxf(m_run[1], mx1);
-        al0 = (n0 == kNegInf || m_run[0] == n0) ? 1.f : exp2f((m_run[0] - n0) * c2);
-        al1 = (n1 == kNegInf || m_run[1] == n1) ? 1.f : exp2f((m_run[1] - n1) * c2);
-        m_run[0] = n0;
-        m_run[1] = n1;
-        // o columns of this lane: heads 2 (t & 1), +1, high (t < 2) or low (t >= 2) half
-        const float b0 = __shfl_xor_sync(kFull, al0, 2), b1 = __shfl_xor_sync(kFull, al1, 2);
-        const float oa0 = t < 2 ? al0 : b0, oa1 = t < 2 ? al1 : b1;
-        if (__any_sync(kFull, oa0 != 1.f || oa1 != 1.f)) {   // a reference moved: rescale o
-#pragma unroll
-            for (int mt = 0; mt < KB; ++mt) {
-                oacc[mt][0] *= oa0; oacc[mt][1] *= oa1;
-                oacc[mt][2] *= oa0; oacc[mt][3] *= oa1;
+            for (int j = 0; j < 4; ++j) {
+                k[j] = (2 * j < D / 16) ? swz_chunk<ROWB>(tk, 2 * j + (m & 1)) : 0u;
+                v[j] = (2 * j < D / 16) ? VOFF + swz_chunk<ROWB>(tv, 2 * j + (lane >> 4)) : 0u;
             }
         }
     }
-    const float p0 = v0 ? exp2f((s[0] - m_run[0]) * c2) : 0.f;
-    const float p1 = v1 ? exp2f((s[1] - m_run[1]) * c2) : 0.f;
-    const float p2 = v2 ? exp2f((s[2] - m_run[0]) * c2) : 0.f;
-    const float p3 = v3 ? exp2f((s[3] - m_run[1]) * c2) : 0.f;
-    l_run[0] = fmaf(l_run[0], al0, p0 + p2);
-    l_run[1] = fmaf(l_run[1], al1, p1 + p3);
-    // P (times V scale / normaliser for FP8) to shared memory, [token][head]
-    float w0 = p0, w1 = p1, w2 = p2, w3 = p3;
-    if constexpr (FP8) {
-        const float fa = svA * vnorm, fb = svB * vnorm;
-        w0 *= fa; w1 *= fa; w2 *= fb; w3 *= fb;
-    }
-    if (t < 2) {
-        *reinterpret_cast<float2*>(&sm_p[g][2 * t]) = make_float2(w0, w1);
-        *reinterpret_cast<float2*>(&sm_p[g + 8][2 * t]) = make_float2(w2, w3);
-    }
-    __syncwarp();
-    // B fragment [P_hi | P_lo]: lane (g, t) holds column g (head g & 3, high half if
-    // g < 4) at the k positions 2t, 2t+1 | 2t+8, 2t+9, i.e. tokens
-    // bf16: 2t, 2t+1 | 2t+8, 2t+9;  FP8 (permuted to the b8 ldmatrix): 4t, 4t+1 | 4t+2, 4t+3
-    const int hc = g & 3;
-    const int ta = FP8 ? 4 * t : 2 * t, tb = FP8 ? 4 * t + 2 : 2 * t + 8;
-    const float e0 = sm_p[ta][hc], e1 = sm_p[ta + 1][hc], e2 = sm_p[tb][hc], e3 = sm_p[tb + 1][hc];
-    uint32_t bb0, bb1;
-    if constexpr (FP8) {
-        const uint32_t h0 = pack_f16(e0, e1), h1 = pack_f16(e2, e3);
-        if (g < 4) {
-            bb0 = h0; bb1 = h1;
-        } else {
-            const __half2 x0 = *reinterpret_cast<const __half2*>(&h0), x1 = *reinterpret_cast<const __half2*>(&h1);
-            bb0 = pack_f16(e0 - __low2float(x0), e1 - __high2float(x0));
-            bb1 = pack_f16(e2 - __low2float(x1), e3 - __high2float(x1));
+};
+
+// ------------------------------------------------------------------ one tile
+struct RowState {
+    float m;     // reference maximum of this lane's head (raw logit units)
+    float l;     // this lane's share of the head's sum of probabilities
+};
+
+// One 16-token tile (tokens t0 .. t0+15 of a segment ending at seg_end) held at
+// shared address `st` (its first ring slot).  qa: the A fragments of the
+// queries (a0, a2 of every k block: rows 0..3 and 4..7 both hold the group's
+// heads, rows 8..15 are zero).  skv/svv: FP8 scales of this lane's tokens 2t, 2t+1,
+// 8+2t, 9+2t (unused for bf16); vnorm: the warp's V-scale normaliser.  hv: this
+// lane's head (g & 3) is real; lo: this lane supplies the low parts of P (g >= 4).
+template <int D, bool FP8, int FMT>
+__device__ __forceinline__ void attend_tile(uint32_t st, const LaneOffsets<D, FP8>& off, int t0, int seg_end,
+                                            bool hv, bool lo, float c2, const float (&skv)[4], const float (&svv)[4],
+                                            float vnorm, float* logit_head, const uint32_t (&qa)[D / 16][2],
+                                            RowState& rs, float (&oacc)[D / 16][4]) {
+    constexpr int KB = D / 16;   // k blocks of QK^T, m-tiles of PV
+    const int lane = threadIdx.x & 31;
+    const int t = lane & 3;
+
+    // ---- S = Qx K^T: n-tile 0 (tokens 0..7) and n-tile 1 (tokens 8..15), kQkChains
+    // independent accumulator chains per n-tile (k blocks dealt round robin)
+    float sa[2][kQkChains][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int c = 0; c < kQkChains; ++c) sa[nt][c][0] = sa[nt][c][1] = sa[nt][c][2] = sa[nt][c][3] = 0.f;
+    if constexpr (!FP8) {
+#pragma unroll
+        for (int kk = 0; kk < KB; ++kk) {
+            uint32_t b[4];   // (b0, b1) of n-tile 0, then of n-tile 1
+            ldsm_x4(b, st + off.k[kk & 3] + (kk >> 2) * 2048);
+            mma16816<false>(sa[0][kk % kQkChains], qa[kk][0], 0u, qa[kk][1], 0u, b[0], b[1]);
+            mma16816<false>(sa[1][kk % kQkChains], qa[kk][0], 0u, qa[kk][1], 0u, b[2], b[3]);
         }
     } else {
-        const uint32_t h0 = pack_bf16(e0, e1), h1 = pack_bf16(e2, e3);
-        if (g < 4) {
-            bb0 = h0; bb1 = h1;
-        } else {
-            const __nv_bfloat162 x0 = *reinterpret_cast<const __nv_bfloat162*>(&h0);
-            const __nv_bfloat162 x1 = *reinterpret_cast<const __nv_bfloat162*>(&h1);
-            bb0 = pack_bf16(e0 - __low2float(x0), e1 - __high2float(x0));
-            bb1 = pack_bf16(e2 - __low2float(x1), e3 - __high2float(x1));
+#pragma unroll
+        for (int j = 0; j < KB / 2; ++j) {
+            uint32_t w[4];   // words: (n-tile 0, k block 2j), (nt 0, 2j+1), (nt 1, 2j), (nt 1, 2j+1)
+            ldsm_x4(w, st + off.k[j]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t b0, b1;
+                fp8x4_to_f16<FMT>(w[q], b0, b1);
+                const int kk = 2 * j + (q & 1);
+                mma16816<true>(sa[q >> 1][kk % kQkChains], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
+            }
         }
-    }
-    // past the segment end the tile holds stale slots or zero fill: P is 0 there,
-    // and a partial tile also zeroes those V elements so that no stale bit pattern
-    // can reach the accumulator (same token order as the B fragment)
-    const bool partial = t0 + 16 > seg_end;   // warp-uniform
-    uint32_t m01 = 0xffffffffu, m23 = 0xffffffffu;
-    if (partial) {
-        m01 = (t0 + ta < seg_end ? 0xffffu : 0u) | (t0 + ta + 1 < seg_end ? 0xffff0000u : 0u);
-        m23 = (t0 + tb < seg_end ? 0xffffu : 0u) | (t0 + tb + 1 < seg_end ? 0xffff0000u : 0u);
     }
 #pragma unroll
-    for (int mt = 0; mt < KB; ++mt) {
-        uint32_t a[4];
-        if constexpr (FP8) {
-            // lanes 0..15 supply token rows 0..15 at dims 16 mt .. 16 mt + 15
-            uint32_t r0, r1;
-            ldsm_b8_trans(r0, r1, vs + swz<ROWB>(lane & 15, 16 * mt));
-            a[0] = e4m3x2_to_f16x2(r0);          // dim g,     tokens 4t, 4t+1
-            a[2] = e4m3x2_to_f16x2(r0 >> 16);    // dim g,     tokens 4t+2, 4t+3
-            a[1] = e4m3x2_to_f16x2(r1);          // dim g + 8, tokens 4t, 4t+1
-            a[3] = e4m3x2_to_f16x2(r1 >> 16);    // dim g + 8, tokens 4t+2, 4t+3
-        } else {
-            // ldmatrix.trans matrix q = lane / 8: tokens 8 (q / 2) + lane % 8, dims 16 mt + 8 (q % 2)
-            const int tok = (lane & 7) + 8 * (lane >> 4);
-            const int byte = 2 * (16 * mt + 8 * ((lane >> 3) & 1));
-            ldsm_x4_trans(a, vs + (byte >> 7) * 2048 + swz<128>(tok, byte & 127));
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int c = 1; c < kQkChains; ++c) { sa[nt][0][0] += sa[nt][c][0]; sa[nt][0][1] += sa[nt][c][1]; }
+    // this lane: head g & 3, tokens 2t, 2t+1 (n-tile 0) and 8+2t, 9+2t (n-tile 1)
+    float s[4] = {sa[0][0][0], sa[0][0][1], sa[1][0][0], sa[1][0][1]};
+    if constexpr (FP8) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[e] *= skv[e];
+    }
+    const int tA = t0 + 2 * t, tB = t0 + 8 + 2 * t;
+    const bool partial = t0 + 16 > seg_end;          // warp-uniform
+    bool v[4] = {hv, hv, hv, hv};
+    if (partial) {
+        v[0] = hv && tA < seg_end; v[1] = hv && tA + 1 < seg_end;
+        v[2] = hv && tB < seg_end; v[3] = hv && tB + 1 < seg_end;
+    }
+    if (hv && !lo) {   // raw logits for the score update, [head][slot]
+        if (!partial || tA + 1 < seg_end) *reinterpret_cast<float2*>(logit_head + tA) = make_float2(s[0], s[1]);
+        else if (tA < seg_end) logit_head[tA] = s[0];
+        if (!partial || tB + 1 < seg_end) *reinterpret_cast<float2*>(logit_head + tB) = make_float2(s[2], s[3]);
+        else if (tB < seg_end) logit_head[tB] = s[2];
+    }
+
+    // ---- online softmax with a lazy reference (moves only past 2^8)
+    float a[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) a[e] = (s[e] - rs.m) * c2;
+    const bool need = (v[0] && a[0] > 8.f) || (v[1] && a[1] > 8.f) || (v[2] && a[2] > 8.f) || (v[3] && a[3] > 8.f);
+    if (__any_sync(kFull, need)) {
+        float mx = fmaxf(fmaxf(v[0] ? s[0] : kNegInf, v[1] ? s[1] : kNegInf),
+                         fmaxf(v[2] ? s[2] : kNegInf, v[3] ? s[3] : kNegInf));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+        const float mn = fmaxf(rs.m, mx);              // uniform over the 4 lanes of a row
+        const float al = (mn == rs.m || rs.m == kNegInf) ? (rs.m == kNegInf ? 0.f : 1.f) : ex2((rs.m - mn) * c2);
+        rs.m = mn;
+        rs.l *= al;
+        // this lane's accumulator columns 2(t & 1), 2(t & 1) + 1 hold heads 2(t & 1), +1:
+        // their factors come from the rows g = 2(t & 1), +1 (lanes 8(t & 1), 8(t & 1) + 4)
+        const float a0 = __shfl_sync(kFull, al, 8 * (t & 1)), a1 = __shfl_sync(kFull, al, 8 * (t & 1) + 4);
+        if (__any_sync(kFull, a0 != 1.f || a1 != 1.f)) {
+#pragma unroll
+            for (int mt = 0; mt < KB; ++mt) {
+                oacc[mt][0] *= a0; oacc[mt][1] *= a1; oacc[mt][2] *= a0; oacc[mt][3] *= a1;
+            }
         }
-        if (partial) {
-            a[0] &= m01; a[1] &= m01; a[2] &= m23; a[3] &= m23;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) a[e] = (s[e] - rs.m) * c2;
+    }
+    float p[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) p[e] = v[e] ? ex2(a[e]) : 0.f;
+    rs.l += (p[0] + p[1]) + (p[2] + p[3]);
+    // the accumulator holds O * vnorm: FP8 tiles fold their V scale in as well
+#pragma unroll
+    for (int e = 0; e < 4; ++e) p[e] *= FP8 ? svv[e] * vnorm : vnorm;
+    // B fragment of [P_hi | P_lo] (column g: head g & 3, high part for g < 4, low part
+    // p - hi for g >= 4) at k = 2t, 2t+1 (b0) and 2t+8, 2t+9 (b1)
+    uint32_t b0, b1;
+    if constexpr (FP8) {
+        const uint32_t h0 = pack_f16(p[0], p[1]), h1 = pack_f16(p[2], p[3]);
+        const __half2 x0 = *reinterpret_cast<const __half2*>(&h0), x1 = *reinterpret_cast<const __half2*>(&h1);
+        b0 = lo ? pack_f16(p[0] - __low2float(x0), p[1] - __high2float(x0)) : h0;
+        b1 = lo ? pack_f16(p[2] - __low2float(x1), p[3] - __high2float(x1)) : h1;
+    } else {
+        const uint32_t h0 = pack_bf16(p[0], p[1]), h1 = pack_bf16(p[2], p[3]);
+        b0 = lo ? pack_bf16(p[0] - bf16_lo(h0), p[1] - bf16_hi(h0)) : h0;
+        b1 = lo ? pack_bf16(p[2] - bf16_lo(h1), p[3] - bf16_hi(h1)) : h1;
+    }
+
+    // ---- O^T += V^T [P_hi | P_lo].  Past the segment end the tile holds stale slots or
+    // zero fill: P is 0 there, and a partial tile also zeroes those V elements so that
+    // no stale bit pattern can reach the accumulator (k = 2t, 2t+1: tokens 2t, 2t+1;
+    // k = 2t+8, 2t+9: tokens 8+2t, 9+2t)
+    uint32_t m0 = 0xffffffffu, m1 = 0xffffffffu;
+    if (partial) {
+        m0 = (tA < seg_end ? 0xffffu : 0u) | (tA + 1 < seg_end ? 0xffff0000u : 0u);
+        m1 = (tB < seg_end ? 0xffffu : 0u) | (tB + 1 < seg_end ? 0xffff0000u : 0u);
+    }
+    if constexpr (!FP8) {
+#pragma unroll
+        for (int mt = 0; mt < KB; ++mt) {
+            uint32_t af[4];   // A fragment of V^T for dims 16 mt .. 16 mt + 15
+            ldsm_x4_trans(af, st + off.v[mt & 3] + (mt >> 2) * 2048);
+            if (partial) { af[0] &= m0; af[1] &= m0; af[2] &= m1; af[3] &= m1; }
+            mma16816<false>(oacc[mt], af[0], af[1], af[2], af[3], b0, b1);
         }
-        mma16816<FP8>(oacc[mt], a, bb0, bb1);
+    } else {
+#pragma unroll
+        for (int j = 0; j < KB / 2; ++j) {
+            uint32_t r[4];   // chunk 2j: dims +g (r0), +8+g (r1); chunk 2j+1: r2, r3
+            ldsm_b8_x2_trans(r, st + off.v[j]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t a0, a2, a1, a3;
+                fp8x4_to_f16<FMT>(r[2 * h], a0, a2);
+                fp8x4_to_f16<FMT>(r[2 * h + 1], a1, a3);
+                if (partial) { a0 &= m0; a1 &= m0; a2 &= m1; a3 &= m1; }
+                mma16816<true>(oacc[2 * j + h], a0, a1, a2, a3, b0, b1);
+            }
+        }
     }
 }
 
-// Q^T B fragments of head g (zero past G) of a row: for block kk, b0 holds the
-// k positions 2t, 2t+1 and b1 2t+8, 2t+9 -- dims 16 kk + (2t, 2t+1 | 2t+8, 2t+9)
-// for bf16 (ldmatrix layout), dims 16 kk + 4t + (0, 1 | 2, 3) in f16 for FP8.
+// A fragments (a0, a2 of every k block) of query row g: head g & 3 (rows 0..3 and
+// 4..7 repeat the group; zero for heads >= G): bf16 in natural dimension order;
+// f16 for FP8 tiles, in the order of the 4-byte K words (dims 16 kk + 4t .. + 3).
 template <int D>
-__device__ __forceinline__ void load_q(const AttnParams& p, int row, bool fp8, uint32_t (&qb)[D / 16][2]) {
-    const int lane = threadIdx.x & 31, fg = lane >> 2, ft = lane & 3;
+__device__ __forceinline__ void load_q(const AttnParams& p, int row, bool fp8, uint32_t (&qa)[D / 16][2]) {
+    const int lane = threadIdx.x & 31, h = (lane >> 2) & 3, t = lane & 3;
     const int b = row / p.d.hkv, gk = row - b * p.d.hkv, G = p.d.G;
-    const bool hv = fg < G;
-    const uint16_t* qrow = p.q + ((size_t)b * p.d.hq + gk * G + (hv ? fg : 0)) * D;
+    const bool hv = h < G;
+    const uint16_t* qrow = p.q + ((size_t)b * p.d.hq + gk * G + (hv ? h : 0)) * D;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
         uint32_t x = 0u, y = 0u;
         if (hv) {
             if (fp8) {
-                const uint2 u = *reinterpret_cast<const uint2*>(qrow + 16 * kk + 4 * ft);
+                const uint2 u = *reinterpret_cast<const uint2*>(qrow + 16 * kk + 4 * t);
                 x = pack_f16(bf16_lo(u.x), bf16_hi(u.x));
                 y = pack_f16(bf16_lo(u.y), bf16_hi(u.y));
             } else {
-                x = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * ft);
-                y = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * ft + 8);
+                x = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * t);
+                y = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * t + 8);
             }
         }
-        qb[kk][0] = x;
-        qb[kk][1] = y;
+        qa[kk][0] = x;
+        qa[kk][1] = y;
     }
 }
 
-template <int D>
-__global__ void __launch_bounds__(32 * kWarps) decode_attn_kernel(const __grid_constant__ AttnParams p) {
+// This CTA's place in the grid: the call runs one wave of P CTAs, shared among the
+// rows in proportion to their lengths.  Row r gets n_r = base(r+1) - base(r) >= 1
+// CTAs, base(r) = r + floor((P - R) Wb(r) / Wtot + 1/2) with Wb(r) the summed
+// lengths (ctx_len of the row's sequence + step + 1) of the rows before it.  Only
+// ctx_len enters, which no CTA modifies, so every CTA derives the same shares.
+struct Share {
+    int row, c, n, base;
+};
+
+__device__ __forceinline__ Share grid_share(const AttnParams& p, int* sm) {
+    const LayerDims& d = p.d;
+    const int lane = threadIdx.x & 31, bid = blockIdx.x, P = gridDim.x;
+    if (threadIdx.x < 32) {
+        const long long extra = P - d.R;   // CTAs beyond one per row
+        long long tot = 0;
+        for (int b0 = 0; b0 < d.batch; b0 += 32) {
+            const int b = b0 + lane;
+            long long L = b < d.batch ? (long long)__ldg(&p.ctx_len[b]) + p.step + 1 : 0;
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) L += __shfl_xor_sync(kFull, L, m);
+            tot += L * d.hkv;
+        }
+        tot = max(tot, 1ll);
+        auto F = [&](long long w) { return (int)((2 * extra * w + tot) / (2 * tot)); };
+        long long run = 0;
+        for (int b0 = 0; b0 < d.batch; b0 += 32) {
+            const int b = b0 + lane;
+            const long long L = b < d.batch ? (long long)__ldg(&p.ctx_len[b]) + p.step + 1 : 0;
+            long long incl = L;
+#pragma unroll
+            for (int m = 1; m < 32; m <<= 1) {
+                const long long y = __shfl_up_sync(kFull, incl, m);
+                if (lane >= m) incl += y;
+            }
+            if (b < d.batch) {
+                long long wb = run + (incl - L) * d.hkv;   // lengths before row (b, 0)
+                for (int g = 0; g < d.hkv; ++g, wb += L) {
+                    const int r = b * d.hkv + g;
+                    const int lo = r + F(wb), hi = r + 1 + F(wb + L);
+                    if (bid >= lo && bid < hi) {
+                        sm[0] = r; sm[1] = bid - lo; sm[2] = hi - lo; sm[3] = lo;
+                    }
+                }
+            }
+            run += __shfl_sync(kFull, incl, 31) * d.hkv;
+        }
+    }
+    __syncthreads();
+    return Share{sm[0], sm[1], sm[2], sm[3]};
+}
+
+// The CTA's tiles: bf16 tiles [a16, e16) then FP8 tiles [a8, e8) of its row, dealt
+// round robin to the warps.  Each warp streams its tiles through its own ring of
+// kSlots slots (a bf16 tile takes two, an FP8 tile one) filled by TMA, then the CTA
+// combines its warps into one (max, sum, unnormalised o) partial in slot blockIdx.x.
+template <int D, int FMT>
+__device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int row, int n16, int n8, int a16,
+                                         int e16, int a8, int e8) {
     using SL = Smem<D>;
     constexpr int KB = D / 16;
-    constexpr int STAGE = SL::kStage;
-    constexpr int VOFF = SL::kTileBytes;
-    constexpr int NB16 = D * 2 / 128;                // bf16 boxes per tile
+    constexpr int SLOT = SL::kSlot;
     const LayerDims& d = p.d;
-    // CTA order, longest work first: the FP8 splits of every row (rows fastest), then
-    // the bf16 splits.  An FP8 split holds twice the tokens of a bf16 split and costs
-    // more per tile, so dispatching it last would leave the longest CTAs in the tail.
-    const int nq = p.nsplit_q * d.R, bid = blockIdx.x;
-    const int row = bid < nq ? bid % d.R : (bid - nq) % d.R;
-    const int split = bid < nq ? p.nsplit_o + bid / d.R : (bid - nq) / d.R;
-    const int b = row / d.hkv, gk = row - b * d.hkv;
-    const int nsplit = p.nsplit_o + p.nsplit_q;
-    const bool fp8 = split >= p.nsplit_o;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int fg = lane >> 2, ft = lane & 3;
-
-    // the split's slot range; the bf16 segment includes the slot of the new token
-    const int n16_old = min(max(p.c.n_bf16[row], 0), d.cap_o);   // counts are clamped to the
-    const bool append = n16_old < d.cap_o;                          // capacities before any use;
-    int s0, s1;                                                     // merge_kernel advances n_bf16
-    if (!fp8) {
-        s0 = split * kSplitBf16;
-        s1 = min(s0 + kSplitBf16, n16_old + (append ? 1 : 0));
-    } else {
-        s0 = (split - p.nsplit_o) * kSplitFp8;
-        s1 = min(s0 + kSplitFp8, min(max(p.c.n_fp8[row], 0), d.cap_q));
-    }
-    if (s0 >= s1) return;                            // nothing live in this split
-
-    extern __shared__ char smem_raw[];
-    char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SL::kBars) + warp * kStages;
-    float (*sm_p)[8] = reinterpret_cast<float (*)[16][8]>(smem + SL::kP)[warp];
-    char* ring = smem + warp * kStages * STAGE;
-    if (lane == 0) {
-#pragma unroll
-        for (int st = 0; st < kStages; ++st) mbar_init(&bars[st], 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    // append: the CTA whose split covers the new slot stores the token before any
-    // tensor load reads that slot (the proxy fence orders the two)
-    if (!fp8 && append && n16_old >= s0 && n16_old < s1) {
-        const uint16_t* kn = p.k_new + ((size_t)b * d.hkv + gk) * D;
-        const uint16_t* vn = p.v_new + ((size_t)b * d.hkv + gk) * D;
-        const size_t sl = (size_t)row * d.cap_o + n16_old;
-        for (int c = tid; c < D / 8; c += blockDim.x) {
-            *reinterpret_cast<uint4*>(p.c.k16 + sl * D + 8 * c) = *reinterpret_cast<const uint4*>(kn + 8 * c);
-            *reinterpret_cast<uint4*>(p.c.v16 + sl * D + 8 * c) = *reinterpret_cast<const uint4*>(vn + 8 * c);
-        }
-        if (tid == 0) {
-            p.c.pos16[sl] = p.ctx_len[b] + p.step;
-            p.c.mu16[sl] = 0.0;
-            p.c.m2_16[sl] = 0.0;
-        }
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-    }
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t ring = sbase + warp * kSlots * SLOT;
+    const uint32_t bars = sbase + SL::kBars + warp * kSlots * 8;
     int* sm_abort = reinterpret_cast<int*>(smem + SL::kAbort);
-    if (tid == 0) *sm_abort = 0;
-    __syncthreads();
 
-    // this warp's tiles: s0 + 16 (warp + 4 i)
-    const int first = s0 + 16 * warp;
-    const int ntiles = first < s1 ? (s1 - first + 16 * kWarps - 1) / (16 * kWarps) : 0;
-    const int ybase = fp8 ? row * d.cap_q : row * d.cap_o;
-    auto issue = [&](int i) {
-        const int st = i % kStages;
-        const int y = ybase + first + 16 * kWarps * i;
-        char* kd = ring + st * STAGE;
-        if (!fp8) {
-            mbar_expect_tx(&bars[st], 2 * 16 * D * 2);
+    // this warp's tiles: list positions warp, warp + 4, ... of [bf16 tiles, FP8 tiles]
+    const int L16 = e16 - a16, L = L16 + (e8 - a8);
+    const int nt16 = L16 > warp ? (L16 - warp + kWarps - 1) / kWarps : 0;
+    const int nt = L > warp ? (L - warp + kWarps - 1) / kWarps : 0;
+    auto tile_of = [&](int i) { const int li = warp + kWarps * i; return li < L16 ? a16 + li : a8 + (li - L16); };
+    // producer state (every lane keeps it; lane 0 issues)
+    int iss = 0, ipos = 0, free_slots = kSlots;
+    auto try_issue = [&]() {
+        while (iss < nt) {
+            const bool bf = iss < nt16;
+            const int sz = bf ? 2 : 1;
+            if (sz > free_slots) break;
+            if (lane == 0) {
+                const uint32_t dst = ring + ipos * SLOT, bar = bars + 8 * ipos;
+                const int jt = tile_of(iss);
+                if (bf) {
+                    const int y = row * d.cap_o + 16 * jt;
+                    mbar_expect_tx(bar, 2 * SLOT);
 #pragma unroll
-            for (int bx = 0; bx < NB16; ++bx) {
-                tma_load_2d(kd + bx * 2048, &p.tm_k16, bx * 64, y, &bars[st]);
-                tma_load_2d(kd + VOFF + bx * 2048, &p.tm_v16, bx * 64, y, &bars[st]);
+                    for (int bx = 0; bx < D * 2 / 128; ++bx) {
+                        tma_load_2d(dst + bx * 2048, &p.tm_k16, bx * 64, y, bar);
+                        tma_load_2d(dst + SLOT + bx * 2048, &p.tm_v16, bx * 64, y, bar);
+                    }
+                } else {
+                    const int y = row * d.cap_q + 16 * jt;
+                    mbar_expect_tx(bar, 2 * 16 * D);
+                    tma_load_2d(dst, &p.tm_k8, 0, y, bar);
+                    tma_load_2d(dst + 16 * D, &p.tm_v8, 0, y, bar);
+                }
             }
-        } else {
-            mbar_expect_tx(&bars[st], 2 * 16 * D);
-            tma_load_2d(kd, &p.tm_k8, 0, y, &bars[st]);
-            tma_load_2d(kd + VOFF, &p.tm_v8, 0, y, &bars[st]);
+            ipos = (ipos + sz) & (kSlots - 1);
+            free_slots -= sz;
+            ++iss;
         }
     };
-    if (lane == 0)
-        for (int i = 0; i < min(kStages, ntiles); ++i) issue(i);
+    try_issue();
 
-    float m_run[2] = {kNegInf, kNegInf}, l_run[2] = {0.f, 0.f}, oacc[KB][4];
+    const int hd = g & 3;                    // this lane's head: rows g and g + 4 repeat it
+    const bool hv = hd < d.G, lo = g >= 4;
+    const float c2 = (float)(p.inv_sqrt_d * 1.4426950408889634);   // log2(e) / sqrt(D)
+    RowState rs{kNegInf, 0.f};
+    float oacc[KB][4];
 #pragma unroll
     for (int mt = 0; mt < KB; ++mt) oacc[mt][0] = oacc[mt][1] = oacc[mt][2] = oacc[mt][3] = 0.f;
-    uint32_t qb[KB][2];
-    load_q<D>(p, row, fp8, qb);
-    const float c2 = (float)(p.inv_sqrt_d * 1.4426950408889634);   // log2(e) / sqrt(D)
+
+    // the largest V scale of the warp's FP8 tiles (1 if it has none); every tile's P is
+    // multiplied by vnorm = 64 / vmax (p < 2^8: p sv vnorm < 2^14, inside f16)
     const float* skb = p.c.sk + (size_t)row * d.cap_q;
     const float* svb = p.c.sv + (size_t)row * d.cap_q;
-    float vmax = 1.f, vnorm = 1.f;                   // FP8: the warp's largest V scale
-    float nskA = 1.f, nskB = 1.f, nsvA = 1.f, nsvB = 1.f;
-    if (fp8) {
-        vmax = 0.f;
-        for (int i = 0; i < ntiles; ++i) {
-            const int tk = first + 16 * kWarps * i + (lane & 15);
-            if (tk < s1) vmax = fmaxf(vmax, __ldg(svb + tk));
-        }
-#pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(kFull, vmax, m));
-        vnorm = vmax > 0.f ? 64.f / vmax : 0.f;   // p < 2^8: p sv vnorm < 2^14, inside f16
-        const int a = min(first + fg, d.cap_q - 1), c = min(first + fg + 8, d.cap_q - 1);
-        nskA = __ldg(skb + a); nskB = __ldg(skb + c);
-        nsvA = __ldg(svb + a); nsvB = __ldg(svb + c);
+    float vmax = 0.f;
+    for (int i = nt16; i < nt; ++i) {
+        const int tk = 16 * tile_of(i) + (lane & 15);
+        if (tk < n8) vmax = fmaxf(vmax, __ldg(svb + tk));
     }
-    float* logit_row = fp8 ? p.logit8 + (size_t)row * d.cap_q * 4 : p.logit16 + (size_t)row * d.cap_o * 4;
-    for (int i = 0; i < ntiles; ++i) {
-        const int st = i % kStages;
-        const int t0 = first + 16 * kWarps * i;
-        if (!mbar_wait(&bars[st], (uint32_t)((i / kStages) & 1))) {
-            // a copy did not land in time: flag it, give every copy this warp issued
-            // (this one included) a last bounded chance to land, and leave the ring
-            // alone from here on (the epilogue below does not reuse it)
-            if (lane == 0) {
-                atomicOr(p.c.status, ARKV_STATUS_TIMEOUT);
-                atomicExch(sm_abort, 1);
-            }
-            for (int j = i; j < min(i + kStages, ntiles); ++j)
-                mbar_wait(&bars[j % kStages], (uint32_t)((j / kStages) & 1));
-            break;
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(kFull, vmax, m));
+    if (!(vmax > 0.f)) vmax = 64.f;
+    const float vnorm = 64.f / vmax;
+
+    int pos = 0;          // ring slot of the next tile to consume
+    uint32_t ph = 0;      // parity of every slot's next phase
+    bool aborted = false;
+    auto wait_tile = [&](int i) -> bool {
+        if (mbar_wait(bars + 8 * pos, (ph >> pos) & 1u)) return true;
+        // a copy did not land in time: flag it, give every copy this warp has in flight
+        // (this one included) a last bounded chance to land, and leave the ring alone
+        if (lane == 0) {
+            atomicOr(p.c.status, ARKV_STATUS_TIMEOUT);
+            atomicExch(sm_abort, 1);
         }
-        const char* ks = ring + st * STAGE;
-        if (!fp8) {
-            attend_tile<D, false>(ks, t0, s1, d.G, c2, 1.f, 1.f, 1.f, 1.f, 1.f, logit_row, qb, m_run, l_run,
-                                  oacc, sm_p);
-        } else {
-            const float skA = nskA, skB = nskB, svA = nsvA, svB = nsvB;
-            if (i + 1 < ntiles) {      // the next tile's scales, one tile ahead
-                const int a = min(t0 + 16 * kWarps + fg, d.cap_q - 1), c = min(t0 + 16 * kWarps + fg + 8, d.cap_q - 1);
-                nskA = __ldg(skb + a); nskB = __ldg(skb + c);
-                nsvA = __ldg(svb + a); nsvB = __ldg(svb + c);
-            }
-            attend_tile<D, true>(ks, t0, s1, d.G, c2, skA, skB, svA, svB, vnorm, logit_row, qb, m_run, l_run,
-                                 oacc, sm_p);
+        uint32_t q = ph;
+        for (int j = i, sp = pos; j < iss; ++j) {
+            mbar_wait(bars + 8 * sp, (q >> sp) & 1u);
+            q ^= 1u << sp;
+            sp = (sp + (j < nt16 ? 2 : 1)) & (kSlots - 1);
         }
+        return false;
+    };
+    auto release = [&](int sz) {
+        ph ^= 1u << pos;
+        pos = (pos + sz) & (kSlots - 1);
+        free_slots += sz;
         __syncwarp();
-        if (lane == 0 && i + kStages < ntiles) {
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            issue(i + kStages);
+        try_issue();
+    };
+
+    // ---- bf16 tiles
+    uint32_t qa[KB][2];
+    if (nt16 > 0) {
+        load_q<D>(p, row, false, qa);
+        const LaneOffsets<D, false> off;
+        float* logit_head = p.logit16 + ((size_t)row * 4 + (hv ? hd : 0)) * p.lstride_o;
+        const float one[4] = {1.f, 1.f, 1.f, 1.f};
+        const int s1 = min(n16, e16 * 16);
+        for (int i = 0; i < nt16; ++i) {
+            if (!wait_tile(i)) { aborted = true; break; }
+            attend_tile<D, false, FMT>(ring + pos * SLOT, off, 16 * tile_of(i), s1, hv, lo, c2, one, one, vnorm,
+                                       logit_head, qa, rs, oacc);
+            release(2);
+        }
+    }
+    // ---- FP8 tiles, their scales loaded one tile ahead
+    if (!aborted && nt > nt16) {
+        load_q<D>(p, row, true, qa);
+        const LaneOffsets<D, true> off;
+        float* logit_head = p.logit8 + ((size_t)row * 4 + (hv ? hd : 0)) * p.lstride_q;
+        const int s1 = min(n8, e8 * 16);
+        float nsk[4], nsv[4];
+        auto load_scales = [&](int t0) {
+            const int tok[4] = {t0 + 2 * t, t0 + 2 * t + 1, t0 + 8 + 2 * t, t0 + 9 + 2 * t};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int k = min(tok[e], d.cap_q - 1);
+                nsk[e] = __ldg(skb + k);
+                nsv[e] = __ldg(svb + k);
+            }
+        };
+        load_scales(16 * tile_of(nt16));
+        for (int i = nt16; i < nt; ++i) {
+            if (!wait_tile(i)) { aborted = true; break; }
+            float skv[4], svv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) { skv[e] = nsk[e]; svv[e] = nsv[e]; }
+            if (i + 1 < nt) load_scales(16 * tile_of(i + 1));
+            attend_tile<D, true, FMT>(ring + pos * SLOT, off, 16 * tile_of(i), s1, hv, lo, c2, skv, svv, vnorm,
+                                      logit_head, qa, rs, oacc);
+            release(1);
         }
     }
 
     __syncthreads();   // every warp has drained its ring: the epilogue may reuse it
-    const size_t pb = (size_t)row * nsplit + split;
+    const size_t pb = blockIdx.x;
     if (*sm_abort) {
         // a wait gave up: copies may still be landing in the ring, so write an empty
         // partial (weight 0 in the merge) without touching shared memory; the status
@@ -518,41 +634,37 @@ __global__ void __launch_bounds__(32 * kWarps) decode_attn_kernel(const __grid_c
             p.part_o[(pb * 4 + idx / D) * D + idx % D] = 0.f;
             if (idx % D == 0) p.part_ml[pb * 4 + idx / D] = make_float2(kNegInf, 0.f);
         }
-        return;
+        return;   // the caller still takes the row's ticket
     }
     float (*sm_o)[4][D] = reinterpret_cast<float (*)[4][D]>(smem + SL::kO);
     float (*sm_m)[4] = reinterpret_cast<float (*)[4]>(smem + SL::kM);
     float (*sm_l)[4] = reinterpret_cast<float (*)[4]>(smem + SL::kL);
     float (*sm_w)[4] = reinterpret_cast<float (*)[4]>(smem + SL::kRed);
     float* sm_max = reinterpret_cast<float*>(smem + SL::kMax);
-    // warp totals.  l: over the lanes sharing a head pair (all fg).  o: oacc[mt] =
-    // (dim 16 mt + fg, columns 2 ft, 2 ft + 1) and (dim 16 mt + fg + 8, same
-    // columns); columns 0..3 hold the high half, 4..7 the low half of heads 0..3.
-    // FP8 partials carry the V-scale normaliser, taken out here.
-#pragma unroll
-    for (int m = 4; m < 32; m <<= 1) {
-        l_run[0] += __shfl_xor_sync(kFull, l_run[0], m);
-        l_run[1] += __shfl_xor_sync(kFull, l_run[1], m);
-    }
-    const float un = fp8 ? vmax * (1.f / 64.f) : 1.f;
+    // warp totals: l of head g over the 4 lanes of row g (rows 4..7 repeat 0..3).  o:
+    // oacc[mt] = O^T at dims 16 mt + g (c0, c1) and 16 mt + g + 8 (c2, c3), columns
+    // 2t, 2t+1; columns 0..3 hold the high part, 4..7 the low part of heads 0..3, so
+    // lanes t and t ^ 2 add up.  The accumulator carries vnorm, taken out here.
+    float l = rs.l;
+    l += __shfl_xor_sync(kFull, l, 1);
+    l += __shfl_xor_sync(kFull, l, 2);
+    const float un = vmax * (1.f / 64.f);
 #pragma unroll
     for (int mt = 0; mt < KB; ++mt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) oacc[mt][e] += __shfl_xor_sync(kFull, oacc[mt][e], 2);
-    if (ft < 2) {
+    if (t < 2) {
 #pragma unroll
         for (int mt = 0; mt < KB; ++mt) {
-            sm_o[warp][2 * ft][16 * mt + fg] = oacc[mt][0] * un;
-            sm_o[warp][2 * ft + 1][16 * mt + fg] = oacc[mt][1] * un;
-            sm_o[warp][2 * ft][16 * mt + fg + 8] = oacc[mt][2] * un;
-            sm_o[warp][2 * ft + 1][16 * mt + fg + 8] = oacc[mt][3] * un;
+            sm_o[warp][2 * t][16 * mt + g] = oacc[mt][0] * un;
+            sm_o[warp][2 * t + 1][16 * mt + g] = oacc[mt][1] * un;
+            sm_o[warp][2 * t][16 * mt + g + 8] = oacc[mt][2] * un;
+            sm_o[warp][2 * t + 1][16 * mt + g + 8] = oacc[mt][3] * un;
         }
-        if (fg == 0) {
-            sm_l[warp][2 * ft] = l_run[0];
-            sm_l[warp][2 * ft + 1] = l_run[1];
-            sm_m[warp][2 * ft] = m_run[0];
-            sm_m[warp][2 * ft + 1] = m_run[1];
-        }
+    }
+    if (g < 4 && t == 0) {
+        sm_l[warp][g] = l;
+        sm_m[warp][g] = rs.m;
     }
     __syncthreads();
     if (tid < 16) {
@@ -579,130 +691,170 @@ __global__ void __launch_bounds__(32 * kWarps) decode_attn_kernel(const __grid_c
     }
 }
 
-// Merges the split partials of one (row, head): M = max of the split maxima,
-// L = sum of l_s exp((m_s - M)/sqrt(D)), o = sum of o_s exp(..) / L.  4 x D
-// threads: thread (q, d) sums the splits s = q mod 4 of output dim d, so every
-// thread has only a few independent loads in flight.  Also publishes (M, L) for
-// the score update.  The row's bf16 count is advanced past the appended token by
-// the last of the row's G merge CTAs to finish (a ticket in the workspace): every
-// merge CTA of the row reads the count it was launched with, so it may only move
-// once all of them have read it.
+// The row's merge, run by the last of its CTAs to finish: M = max of the partial
+// maxima, L = sum of l_s exp((m_s - M)/sqrt(D)), o = sum of o_s exp(..) / L over
+// the row's partials (slots base .. base + n - 1), for every head of the group,
+// one warp per head (lane l owns dims 4l .. 4l+3 for D = 128, 2l, 2l+1 for D = 64).
+// Each lane weighs the partials l, l + 32, ..., and the weights reach the other
+// lanes by shuffles.  Publishes (M, L) for the score update.
 template <int D>
-__global__ void __launch_bounds__(4 * D) merge_kernel(const AttnParams p) {
+__device__ __forceinline__ void row_merge(const AttnParams& p, int row, int base, int n) {
+    constexpr int VEC = D / 32;
     const LayerDims& d = p.d;
-    const int row = blockIdx.x, h = blockIdx.y;
-    const int b = row / d.hkv, g = row - b * d.hkv;
-    const int nsplit = p.nsplit_o + p.nsplit_q;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    extern __shared__ float sm_w[];                  // [nlive] weights, then [4][D] partial sums
-    __shared__ float sm_red[4 * D / 32];
-    __shared__ float sm_ML[2];
-    const double inv = p.inv_sqrt_d;
-    // the live splits of the row: j < nlo -> bf16 split j, else fp8 split j - nlo
-    const int n16_old = min(max(p.c.n_bf16[row], 0), d.cap_o);
-    const int nl16 = n16_old + (n16_old < d.cap_o ? 1 : 0);
-    const int n8 = min(max(p.c.n_fp8[row], 0), d.cap_q);
-    const int nlo = (nl16 + kSplitBf16 - 1) / kSplitBf16, nlive = nlo + (n8 + kSplitFp8 - 1) / kSplitFp8;
-    auto split_of = [&](int j) { return j < nlo ? j : p.nsplit_o + (j - nlo); };
-    const float2* pml = p.part_ml + (size_t)row * nsplit * 4;
-    // the partial outputs this thread sums (splits q, q + 4, ...) do not depend on
-    // the weights: their loads are issued first, so their latency overlaps the
-    // reductions below
-    const int q = tid / D, dd = tid - q * D;
-    const float* po = p.part_o + (size_t)row * nsplit * 4 * D + (size_t)h * D + dd;
-    constexpr int kPre = 12;
-    float pre[kPre];
+    const int lane = threadIdx.x & 31, h = threadIdx.x >> 5;
+    if (h >= d.G) return;
+    const int b = row / d.hkv, gk = row - b * d.hkv;
+    const float2* pml = p.part_ml + (size_t)base * 4 + h;
+    const float* po = p.part_o + ((size_t)base * 4 + h) * D + VEC * lane;
+    float M = kNegInf;
+    for (int j = lane; j < n; j += 32) M = fmaxf(M, __ldcg(pml + (size_t)j * 4).x);
 #pragma unroll
-    for (int k = 0; k < kPre; ++k) {
-        const int sidx = q + 4 * k;
-        pre[k] = sidx < nlive ? po[(size_t)split_of(sidx) * 4 * D] : 0.f;
+    for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, m));
+    float L = 0.f, acc[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+    for (int j0 = 0; j0 < n; j0 += 32) {
+        float wl = 0.f;
+        if (j0 + lane < n) {
+            const float2 ml = __ldcg(pml + (size_t)(j0 + lane) * 4);
+            wl = (ml.y > 0.f && M != kNegInf) ? exp_scaled(ml.x, M, p.inv_sqrt_d) : 0.f;
+            L = fmaf(ml.y, wl, L);
+        }
+        const int cnt = min(32, n - j0);
+#pragma unroll 8
+        for (int q = 0; q < cnt; ++q) {
+            const float w = __shfl_sync(kFull, wl, q);
+            const float* src = po + (size_t)(j0 + q) * 4 * D;
+            if constexpr (VEC == 4) {
+                const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
+                acc[0] = fmaf(v.x, w, acc[0]); acc[1] = fmaf(v.y, w, acc[1]);
+                acc[2] = fmaf(v.z, w, acc[2]); acc[3] = fmaf(v.w, w, acc[3]);
+            } else {
+                const float2 v = __ldcg(reinterpret_cast<const float2*>(src));
+                acc[0] = fmaf(v.x, w, acc[0]); acc[1] = fmaf(v.y, w, acc[1]);
+            }
+        }
+    }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) L += __shfl_xor_sync(kFull, L, m);
+    float* out = p.o + ((size_t)b * d.hq + gk * d.G + h) * D + VEC * lane;
+    const float inv = 1.f / L;
+    if constexpr (VEC == 4)
+        *reinterpret_cast<float4*>(out) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    else
+        *reinterpret_cast<float2*>(out) = make_float2(acc[0] * inv, acc[1] * inv);
+    if (lane == 0) p.ml[(size_t)row * 4 + h] = make_float2(M, L);
+}
+
+template <int D, int FMT>
+__global__ void __launch_bounds__(32 * kWarps, ARKV_MIN_CTAS) decode_attn_kernel(const __grid_constant__ AttnParams p) {
+    using SL = Smem<D>;
+    const LayerDims& d = p.d;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ unsigned sm_ticket;
+    extern __shared__ char smem_raw[];
+    char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const Share sh = grid_share(p, reinterpret_cast<int*>(smem + SL::kShare));
+    const int row = sh.row, b = row / d.hkv, gk = row - b * d.hkv;
+
+    // the row's counts, read once by every CTA of the row; the last one to finish
+    // advances n_bf16, so no CTA of the row can see the advanced count
+    const int n16_old = min(max(p.c.n_bf16[row], 0), d.cap_o);   // counts are clamped to the
+    const int n8 = min(max(p.c.n_fp8[row], 0), d.cap_q);          // capacities before any use
+    const bool append = n16_old < d.cap_o;
+    const int n16 = n16_old + (append ? 1 : 0);                    // the new token included
+    // this CTA's share of the row, in units of 16-token FP8 tiles (a bf16 tile counts
+    // two): tile j of bf16 starts at unit 2j, FP8 tile j at 2 T16 + j; the CTA takes
+    // the tiles starting in [u0, u1)
+    const int T16 = (n16 + 15) / 16, T8 = (n8 + 15) / 16, U = 2 * T16 + T8;
+    const int u0 = (int)((long long)U * sh.c / sh.n), u1 = (int)((long long)U * (sh.c + 1) / sh.n);
+    const int a16 = min((u0 + 1) / 2, T16), e16 = min((u1 + 1) / 2, T16);
+    const int a8 = min(max(u0 - 2 * T16, 0), T8), e8 = min(max(u1 - 2 * T16, 0), T8);
+
+    if (e16 > a16 || e8 > a8) {
+        if (lane == 0) {
+            const uint32_t bars = smem_u32(smem + SL::kBars) + warp * kSlots * 8;
+#pragma unroll
+            for (int st = 0; st < kSlots; ++st) mbar_init(bars + 8 * st, 1);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        }
+        // append: the CTA whose tiles cover the new slot stores the token before any
+        // tensor load reads that slot (the proxy fence orders the two)
+        if (append && n16_old >= 16 * a16 && n16_old < 16 * e16) {
+            const uint16_t* kn = p.k_new + ((size_t)b * d.hkv + gk) * D;
+            const uint16_t* vn = p.v_new + ((size_t)b * d.hkv + gk) * D;
+            const size_t sl = (size_t)row * d.cap_o + n16_old;
+            for (int c = tid; c < D / 8; c += blockDim.x) {
+                *reinterpret_cast<uint4*>(p.c.k16 + sl * D + 8 * c) = *reinterpret_cast<const uint4*>(kn + 8 * c);
+                *reinterpret_cast<uint4*>(p.c.v16 + sl * D + 8 * c) = *reinterpret_cast<const uint4*>(vn + 8 * c);
+            }
+            if (tid == 0) {
+                p.c.pos16[sl] = p.ctx_len[b] + p.step;
+                p.c.mu16[sl] = 0.0;
+                p.c.m2_16[sl] = 0.0;
+            }
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
+        if (tid == 0) *reinterpret_cast<int*>(smem + SL::kAbort) = 0;
+        __syncthreads();
+        cta_body<D, FMT>(p, smem, row, n16, n8, a16, e16, a8, e8);
+    } else {
+        for (int idx = tid; idx < 4 * D; idx += blockDim.x) {   // nothing to attend: an empty partial
+            p.part_o[(size_t)blockIdx.x * 4 * D + idx] = 0.f;
+            if (idx < 4) p.part_ml[(size_t)blockIdx.x * 4 + idx] = make_float2(kNegInf, 0.f);
+        }
     }
 
-    float mloc = kNegInf;
-    for (int s = tid; s < nlive; s += blockDim.x) mloc = fmaxf(mloc, pml[split_of(s) * 4 + h].x);
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(kFull, mloc, m));
-    if (lane == 0) sm_red[warp] = mloc;
+    // the row's ticket: every CTA of the row takes one after its partial is visible;
+    // the last one merges and moves the row's bf16 count
+    __threadfence();
     __syncthreads();
+    if (tid == 0) sm_ticket = atomicAdd(&p.counter[row], 1u);
+    __syncthreads();
+    if (sm_ticket != (unsigned)(sh.n - 1)) return;
+    __threadfence();
+    row_merge<D>(p, row, sh.base, sh.n);
     if (tid == 0) {
-        float M = kNegInf;
-        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) M = fmaxf(M, sm_red[w]);
-        sm_ML[0] = M;
-    }
-    __syncthreads();
-    const float M = sm_ML[0];
-    float lloc = 0.f;
-    for (int s = tid; s < nlive; s += blockDim.x) {
-        const float2 ml = pml[split_of(s) * 4 + h];
-        const float wt = (ml.y > 0.f && M != kNegInf) ? exp_scaled(ml.x, M, inv) : 0.f;
-        sm_w[s] = wt;
-        lloc = fmaf(ml.y, wt, lloc);
-    }
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) lloc += __shfl_xor_sync(kFull, lloc, m);
-    __syncthreads();
-    if (lane == 0) sm_red[warp] = lloc;
-    __syncthreads();
-    if (tid == 0) {
-        float L = 0.f;
-        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) L += sm_red[w];
-        sm_ML[1] = L;
-        p.ml[(size_t)row * 4 + h] = make_float2(M, L);
-    }
-    __syncthreads();   // the weights
-    float acc = 0.f;
-#pragma unroll
-    for (int k = 0; k < kPre; ++k) {
-        const int sidx = q + 4 * k;
-        if (sidx < nlive && sm_w[sidx] != 0.f) acc = fmaf(pre[k], sm_w[sidx], acc);
-    }
-#pragma unroll 4
-    for (int s = q + 4 * kPre; s < nlive; s += 4) {
-        const float wt = sm_w[s];
-        if (wt != 0.f) acc = fmaf(po[(size_t)split_of(s) * 4 * D], wt, acc);
-    }
-    float* sm_acc = sm_w + nsplit;
-    sm_acc[q * D + dd] = acc;
-    __syncthreads();
-    if (q == 0 && h < d.G) {
-        const float o = (sm_acc[dd] + sm_acc[D + dd]) + (sm_acc[2 * D + dd] + sm_acc[3 * D + dd]);
-        p.o[((size_t)b * d.hq + g * d.G + h) * D + dd] = o / sm_ML[1];
-    }
-    if (tid == 0) {
-        __threadfence();                                 // this CTA's reads of the count come first
-        if (atomicAdd(&p.counter[row], 1u) == (unsigned)(d.G - 1)) {
-            p.counter[row] = 0u;                         // ready for the next call
-            if (n16_old < d.cap_o) p.c.n_bf16[row] = n16_old + 1;
-            else atomicOr(p.c.status, ARKV_STATUS_BF16_FULL);   // the new token was dropped
-        }
+        p.counter[row] = 0u;                                   // ready for the next call
+        if (append) p.c.n_bf16[row] = n16_old + 1;
+        else atomicOr(p.c.status, ARKV_STATUS_BF16_FULL);      // the new token was dropped
     }
 }
 
 // One thread per live slot: x = sum over the group's heads of exp((raw - M)/sqrt(D)) / L,
-// then one Welford step with the token's observation count.
+// then one Welford step with the token's observation count (float64 state).
 __global__ void __launch_bounds__(256) score_update_kernel(const ScoreParams p) {
     const LayerDims& d = p.d;
     const int row = blockIdx.y, b = row / d.hkv;
-    __shared__ float2 sml[4];   // final (max, sum) of every head
-    if (threadIdx.x < 4) sml[threadIdx.x] = __ldg(&p.ml[(size_t)row * 4 + threadIdx.x]);
+    __shared__ float sm_m[4];
+    __shared__ double sm_il[4];   // 1 / L of every head
+    if (threadIdx.x < 4) {
+        const float2 ml = __ldg(&p.ml[(size_t)row * 4 + threadIdx.x]);
+        sm_m[threadIdx.x] = ml.x;
+        sm_il[threadIdx.x] = 1.0 / (double)ml.y;
+    }
     __syncthreads();
     const int n16 = min(max(__ldg(&p.c.n_bf16[row]), 0), d.cap_o);
     const int n8 = min(max(__ldg(&p.c.n_fp8[row]), 0), d.cap_q);
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n16 + n8) return;
     const bool bf = i < n16;
-    const size_t sl = bf ? (size_t)row * d.cap_o + i : (size_t)row * d.cap_q + (i - n16);
-    const float4 lg = __ldg(bf ? reinterpret_cast<const float4*>(p.logit16) + sl
-                               : reinterpret_cast<const float4*>(p.logit8) + sl);
+    const int slot = bf ? i : i - n16;
+    const size_t sl = bf ? (size_t)row * d.cap_o + slot : (size_t)row * d.cap_q + slot;
+    const float* lg = bf ? p.logit16 + (size_t)row * 4 * p.lstride_o + slot
+                         : p.logit8 + (size_t)row * 4 * p.lstride_q + slot;
+    const size_t hs = bf ? p.lstride_o : p.lstride_q;
     const int pos = __ldg(bf ? p.c.pos16 + sl : p.c.pos8 + sl);
     double* __restrict__ mu = bf ? p.c.mu16 + sl : p.c.mu8 + sl;
     double* __restrict__ m2 = bf ? p.c.m2_16 + sl : p.c.m2_8 + sl;
+    float raw[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) raw[h] = h < d.G ? __ldg(lg + h * hs) : 0.f;
     const double mu_old = *mu, m2_old = *m2;
-    const float lv[4] = {lg.x, lg.y, lg.z, lg.w};
     double x = 0.0;
 #pragma unroll
     for (int h = 0; h < 4; ++h)
-        if (h < d.G) x += (double)exp_scaled(lv[h], sml[h].x, p.inv_sqrt_d) / (double)sml[h].y;
+        if (h < d.G) x += (double)exp_scaled(raw[h], sm_m[h], p.inv_sqrt_d) * sm_il[h];
     const int n = obs_count_after(pos, __ldg(&p.ctx_len[b]), p.step, d.n_obs);
     double mv = mu_old, qv = m2_old;
     const double dl = x - mv;
@@ -744,17 +896,17 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem
 
 DecodeWs decode_ws_layout(const LayerDims& d) {
     DecodeWs w{};
-    w.nsplit_o = (d.cap_o + kSplitBf16 - 1) / kSplitBf16;
-    w.nsplit_q = (d.cap_q + kSplitFp8 - 1) / kSplitFp8;
-    const size_t ns = (size_t)(w.nsplit_o + w.nsplit_q);
+    w.parts = d.R > kMaxGrid ? d.R : kMaxGrid;
+    w.lstride_o = (d.cap_o + 3) & ~3;   // logit rows padded to 16 bytes
+    w.lstride_q = (d.cap_q + 3) & ~3;
     auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
     size_t off = 0;
     w.counter = off; off = al(off + sizeof(unsigned) * d.R);
     w.ml = off;      off = al(off + sizeof(float2) * d.R * 4);
-    w.part_ml = off; off = al(off + sizeof(float2) * d.R * ns * 4);
-    w.part_o = off;  off = al(off + sizeof(float) * d.R * ns * 4 * d.D);
-    w.logit16 = off; off = al(off + sizeof(float) * 4 * (size_t)d.R * d.cap_o);
-    w.logit8 = off;  off = al(off + sizeof(float) * 4 * (size_t)d.R * d.cap_q);
+    w.part_ml = off; off = al(off + sizeof(float2) * (size_t)w.parts * 4);
+    w.part_o = off;  off = al(off + sizeof(float) * (size_t)w.parts * 4 * d.D);
+    w.logit16 = off; off = al(off + sizeof(float) * 4 * (size_t)d.R * w.lstride_o);
+    w.logit8 = off;  off = al(off + sizeof(float) * 4 * (size_t)d.R * w.lstride_q);
     w.total = off;
     return w;
 }
@@ -771,24 +923,40 @@ cudaError_t launch_decode_attn(AttnParams& p, cudaStream_t s) {
                     make_map(&p.tm_v8, p.c.v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D, (long long)d.R * d.cap_q, D,
                              D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
     if (!ok) return cudaErrorInvalidValue;
-    const int nsplit = p.nsplit_o + p.nsplit_q;
-    const dim3 mgrid(d.R, d.G);
-    const size_t mdyn = sizeof(float) * ((size_t)nsplit + 4 * (size_t)D);
-    if (mdyn > 48 * 1024) return cudaErrorInvalidValue;
-    static unsigned char done128[64], done64[64];
-    if ((long long)nsplit * d.R > 0x7fffffffLL) return cudaErrorInvalidValue;
-    const dim3 grid(nsplit * d.R);   // one CTA per (split, row); order set in the kernel
-    if (D == 128) {
-        const cudaError_t e = allow_max_dyn_smem(decode_attn_kernel<128>, done128);
-        if (e != cudaSuccess) return e;
-        decode_attn_kernel<128><<<grid, 32 * kWarps, Smem<128>::kBytes, s>>>(p);
-        merge_kernel<128><<<mgrid, 4 * 128, mdyn, s>>>(p);
-    } else {
-        const cudaError_t e = allow_max_dyn_smem(decode_attn_kernel<64>, done64);
-        if (e != cudaSuccess) return e;
-        decode_attn_kernel<64><<<grid, 32 * kWarps, Smem<64>::kBytes, s>>>(p);
-        merge_kernel<64><<<mgrid, 4 * 64, mdyn, s>>>(p);
-    }
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    static unsigned char done[4][64];
+    static int resident[4][64];   // CTAs of the kernel one SM holds, per device
+    static int sms[64];
+    auto go = [&](auto kernel, int which, int bytes) {
+        cudaError_t err = allow_max_dyn_smem(kernel, done[which]);
+        if (err != cudaSuccess) return err;
+        if (dev < 64 && resident[which][dev] == 0) {
+            int n = 0, m = 0;
+            if ((err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, 32 * kWarps, bytes)) != cudaSuccess)
+                return err;
+            if ((err = cudaDeviceGetAttribute(&m, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
+            sms[dev] = m;
+            resident[which][dev] = n > 0 ? n : 1;
+        }
+        // one wave of CTAs, at most one per 16 units (eight bf16 tiles) of the largest
+        // cache, at least one per row
+        const long long units = (long long)d.R * (2 * ((d.cap_o + 16) / 16) + (d.cap_q + 15) / 16);
+        long long P = dev < 64 ? (long long)sms[dev] * resident[which][dev] : 444;
+        P = P < units / 16 ? P : units / 16;
+        if (P > kMaxGrid) P = kMaxGrid;
+        if (P < d.R) P = d.R;
+        kernel<<<dim3((unsigned)P), 32 * kWarps, bytes, s>>>(p);
+        return cudaSuccess;
+    };
+    if (D == 128)
+        e = d.fmt == ARKV_FMT_E5M2 ? go(decode_attn_kernel<128, ARKV_FMT_E5M2>, 0, Smem<128>::kBytes)
+                                   : go(decode_attn_kernel<128, ARKV_FMT_E4M3>, 1, Smem<128>::kBytes);
+    else
+        e = d.fmt == ARKV_FMT_E5M2 ? go(decode_attn_kernel<64, ARKV_FMT_E5M2>, 2, Smem<64>::kBytes)
+                                   : go(decode_attn_kernel<64, ARKV_FMT_E4M3>, 3, Smem<64>::kBytes);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -23,11 +23,15 @@ namespace {
 
 constexpr int kSmemKeyLimit = 24 * 1024;   // 8-byte keys kept in shared memory up to this many slots
 
+constexpr int kCand = 2048;                 // candidate list of a radix selection, once it is this small
+
 struct RowShared {
     unsigned hist[256];
-    int warp_sum[32];
+    int warp_sum[33];
     int sel[4];
     int misc[16];
+    int ncand;
+    int cand[kCand];
 };
 
 // ------------------------------------------------------------------ block helpers
@@ -45,48 +49,48 @@ __device__ __forceinline__ int block_sum(int v, RowShared& sh) {
     return t;
 }
 
-// Exclusive prefix sum of one int per thread over the block; *total = block sum.
-__device__ __forceinline__ int block_excl_scan(int v, int* total, RowShared& sh) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    int x = v;
-#pragma unroll
-    for (int m = 1; m < 32; m <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, m);
-        if (lane >= m) x += y;
-    }
-    __syncthreads();
-    if (lane == 31) sh.warp_sum[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        int w = lane < nw ? sh.warp_sum[lane] : 0;
-#pragma unroll
-        for (int m = 1; m < 32; m <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, w, m);
-            if (lane >= m) w += y;
-        }
-        sh.warp_sum[lane] = w;   // inclusive over warps
-    }
-    __syncthreads();
-    const int before = warp > 0 ? sh.warp_sum[warp - 1] : 0;
-    *total = sh.warp_sum[nw - 1];
-    __syncthreads();
-    return before + x - v;
-}
-
 // Calls f(i, rank) for every i in [begin, end) with pred(i), rank = number of
-// earlier such i.  Returns the count.  All threads must call it.
+// earlier such i.  Returns the count.  All threads must call it.  Each warp owns a
+// contiguous chunk of the range: it counts its chunk (ballots), one block scan of
+// the warps' counts gives every warp its first rank, and a second walk over the
+// chunk emits in order.
 template <class Pred, class F>
 __device__ int block_enumerate(int begin, int end, Pred pred, F f, RowShared& sh) {
-    int running = 0;
-    for (int base = begin; base < end; base += blockDim.x) {
-        const int i = base + threadIdx.x;
-        const int flag = (i < end && pred(i)) ? 1 : 0;
-        int total;
-        const int excl = block_excl_scan(flag, &total, sh);
-        if (flag) f(i, running + excl);
-        running += total;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int n = max(end - begin, 0);
+    const int chunk = (((n + nw - 1) / nw) + 31) & ~31;
+    const int c0 = begin + warp * chunk, c1 = min(c0 + chunk, end);
+    int cnt = 0;
+    for (int i0 = c0; i0 < c1; i0 += 32) {
+        const int i = i0 + lane;
+        cnt += __popc(__ballot_sync(0xffffffffu, i < c1 && pred(i)));
     }
-    return running;
+    __syncthreads();                       // earlier users of warp_sum are done
+    if (lane == 0) sh.warp_sum[warp] = cnt;
+    __syncthreads();
+    if (warp == 0) {
+        const int v = lane < nw ? sh.warp_sum[lane] : 0;
+        int x = v;
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, m);
+            if (lane >= m) x += y;
+        }
+        sh.warp_sum[lane] = x - v;         // exclusive
+        if (lane == 31) sh.warp_sum[32] = x;
+    }
+    __syncthreads();
+    int off = sh.warp_sum[warp];
+    const int total = sh.warp_sum[32];
+    for (int i0 = c0; i0 < c1; i0 += 32) {
+        const int i = i0 + lane;
+        const bool fl = i < c1 && pred(i);
+        const unsigned bal = __ballot_sync(0xffffffffu, fl);
+        if (fl) f(i, off + __popc(bal & ((1u << lane) - 1u)));
+        off += __popc(bal);
+    }
+    __syncthreads();
+    return total;
 }
 
 template <class Pred>
@@ -109,20 +113,40 @@ __device__ __forceinline__ bool sel_in(const Sel& s, uint64_t key, int pos) {
     return key > s.cut || (key == s.cut && (s.all_ties || pos <= s.pos_max));
 }
 
+// One histogram update per group of lanes holding the same digit.
+__device__ __forceinline__ void hist_add(unsigned* hist, bool valid, unsigned digit) {
+    const unsigned peers = __match_any_sync(0xffffffffu, valid ? digit : 0x100u);
+    if (valid && (threadIdx.x & 31) == (unsigned)(__ffs(peers) - 1)) atomicAdd(&hist[digit], (unsigned)__popc(peers));
+}
+
 // k-th largest key (of unsigned type KT) among eligible elements (1 <= k <= count):
 // returns cut and, through need/eq, how many of the elements equal to cut are
-// taken / exist.
+// taken / exist.  8-bit digits from the top; once the elements that share the
+// prefix found so far number at most kCand, they are gathered into a list and the
+// remaining digits are taken over the list only.
 template <class KT, class KeyF, class Elig>
 __device__ KT radix_kth(KeyF key, Elig elig, int n, int k, int* need, int* eq, RowShared& sh) {
     KT prefix = 0, pmask = 0;
-    int kk = k, last_eq = 0;
+    int kk = k, last_eq = 0, nl = -1;       // nl >= 0: the candidates are listed
     for (int shift = 8 * (int)sizeof(KT) - 8; shift >= 0; shift -= 8) {
         for (int i = threadIdx.x; i < 256; i += blockDim.x) sh.hist[i] = 0;
         __syncthreads();
-        for (int i = threadIdx.x; i < n; i += blockDim.x) {
-            if (!elig(i)) continue;
-            const KT kv = key(i);
-            if ((kv & pmask) == prefix) atomicAdd(&sh.hist[(unsigned)(kv >> shift) & 255u], 1u);
+        if (nl < 0) {
+            for (int base = 0; base < n; base += blockDim.x) {
+                const int i = base + threadIdx.x;
+                bool v = i < n && elig(i);
+                KT kv = 0;
+                if (v) { kv = key(i); v = (kv & pmask) == prefix; }
+                hist_add(sh.hist, v, (unsigned)(kv >> shift) & 255u);
+            }
+        } else {
+            for (int base = 0; base < nl; base += blockDim.x) {
+                const int j = base + threadIdx.x;
+                bool v = j < nl;
+                KT kv = 0;
+                if (v) { kv = key(sh.cand[j]); v = (kv & pmask) == prefix; }
+                hist_add(sh.hist, v, (unsigned)(kv >> shift) & 255u);
+            }
         }
         __syncthreads();
         if (threadIdx.x < 32) {
@@ -153,6 +177,7 @@ __device__ KT radix_kth(KeyF key, Elig elig, int n, int k, int* need, int* eq, R
                     above += cnt[j];
                 }
             }
+            if (lane == 0) sh.ncand = 0;
         }
         __syncthreads();
         const KT bin = (KT)sh.sel[0];
@@ -160,6 +185,20 @@ __device__ KT radix_kth(KeyF key, Elig elig, int n, int k, int* need, int* eq, R
         last_eq = sh.sel[2];
         prefix |= bin << shift;
         pmask |= (KT)0xff << shift;
+        if (nl < 0 && shift > 0 && last_eq <= kCand) {
+            // gather the elements that share the prefix (any order: only counts follow)
+            for (int base = 0; base < n; base += blockDim.x) {
+                const int i = base + threadIdx.x;
+                const bool v = i < n && elig(i) && (key(i) & pmask) == prefix;
+                const unsigned bal = __ballot_sync(0xffffffffu, v);
+                int slot0 = 0;
+                if ((threadIdx.x & 31) == 0 && bal) slot0 = atomicAdd(&sh.ncand, __popc(bal));
+                slot0 = __shfl_sync(0xffffffffu, slot0, 0);
+                if (v) sh.cand[slot0 + __popc(bal & ((1u << (threadIdx.x & 31)) - 1u))] = i;
+            }
+            __syncthreads();
+            nl = sh.ncand;
+        }
         __syncthreads();
     }
     *need = kk;
@@ -211,16 +250,18 @@ __device__ __forceinline__ void warp_copy_fp8_row(uint8_t* dst, const uint8_t* s
         reinterpret_cast<uint2*>(dst)[w] = reinterpret_cast<const uint2*>(src)[w];
 }
 
-// Quantize one bf16 row (D elements) held in global memory into codes + scale.
+// Quantize one bf16 row (D elements) held in global memory into codes + scale, in
+// the layer's FP8 format.
 template <int D>
-__device__ __forceinline__ float warp_quantize_row(const uint16_t* src, uint8_t* dst) {
+__device__ __forceinline__ float warp_quantize_row(const uint16_t* src, uint8_t* dst, int fmt) {
     constexpr int EPL = D / 32;
     const int lane = threadIdx.x & 31;
     float x[EPL];
 #pragma unroll
     for (int e = 0; e < EPL; ++e) x[e] = bf16_to_f32(src[lane * EPL + e]);
     uint8_t c[EPL];
-    const float s = quantize_warp<EPL>(x, c);
+    const float s = fmt == ARKV_FMT_E5M2 ? quantize_warp<EPL, ARKV_FMT_E5M2>(x, c)
+                                         : quantize_warp<EPL, ARKV_FMT_E4M3>(x, c);
 #pragma unroll
     for (int e = 0; e < EPL; ++e) dst[lane * EPL + e] = c[e];
     return s;
@@ -359,8 +400,8 @@ __global__ void __launch_bounds__(kRowThreads) reassign_kernel(const ReassignPar
     __syncthreads();
     for (int r = warp; r < n_dem; r += nwarps) {
         const int src = src_list[r], dst = hole_list[n_mov8 + r];
-        const float skv = warp_quantize_row<D>(p.c.k16 + (b16 + src) * D, p.c.k8 + (b8 + dst) * D);
-        const float svv = warp_quantize_row<D>(p.c.v16 + (b16 + src) * D, p.c.v8 + (b8 + dst) * D);
+        const float skv = warp_quantize_row<D>(p.c.k16 + (b16 + src) * D, p.c.k8 + (b8 + dst) * D, d.fmt);
+        const float svv = warp_quantize_row<D>(p.c.v16 + (b16 + src) * D, p.c.v8 + (b8 + dst) * D, d.fmt);
         if ((tid & 31) == 0) {
             p.c.sk[b8 + dst] = skv;
             p.c.sv[b8 + dst] = svv;
@@ -468,8 +509,8 @@ __global__ void __launch_bounds__(kRowThreads) pack_kernel(const PackParams p) {
             }
         } else {
             if (r >= d.cap_q) continue;
-            const float skv = warp_quantize_row<D>(ks, p.c.k8 + (b8 + r) * D);
-            const float svv = warp_quantize_row<D>(vs, p.c.v8 + (b8 + r) * D);
+            const float skv = warp_quantize_row<D>(ks, p.c.k8 + (b8 + r) * D, d.fmt);
+            const float svv = warp_quantize_row<D>(vs, p.c.v8 + (b8 + r) * D, d.fmt);
             if ((tid & 31) == 0) {
                 p.c.sk[b8 + r] = skv;
                 p.c.sv[b8 + r] = svv;
@@ -485,16 +526,16 @@ __global__ void __launch_bounds__(kRowThreads) pack_kernel(const PackParams p) {
     }
 }
 
+template <int FMT>
 __global__ void fp8_encode_kernel(const float* x, uint8_t* out, size_t n) {
+    constexpr __nv_fp8_interpretation_t kInterp = FMT == ARKV_FMT_E5M2 ? __NV_E5M2 : __NV_E4M3;
     const size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 2;
     if (i + 1 < n) {
-        const __nv_fp8x2_storage_t c =
-            __nv_cvt_float2_to_fp8x2(make_float2(x[i], x[i + 1]), __NV_SATFINITE, __NV_E4M3);
+        const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(make_float2(x[i], x[i + 1]), __NV_SATFINITE, kInterp);
         out[i] = (uint8_t)(c & 0xff);
         out[i + 1] = (uint8_t)(c >> 8);
     } else if (i < n) {
-        const __nv_fp8x2_storage_t c =
-            __nv_cvt_float2_to_fp8x2(make_float2(x[i], 0.f), __NV_SATFINITE, __NV_E4M3);
+        const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(make_float2(x[i], 0.f), __NV_SATFINITE, kInterp);
         out[i] = (uint8_t)(c & 0xff);
     }
 }
@@ -540,11 +581,12 @@ cudaError_t launch_quantize_pack(const PackParams& p, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_fp8_encode(const float* x, uint8_t* out, size_t n, cudaStream_t s) {
+cudaError_t launch_fp8_encode(int fmt, const float* x, uint8_t* out, size_t n, cudaStream_t s) {
     if (n == 0) return cudaSuccess;
     const size_t pairs = (n + 1) / 2;
     const unsigned blocks = (unsigned)((pairs + 255) / 256);
-    fp8_encode_kernel<<<blocks, 256, 0, s>>>(x, out, n);
+    if (fmt == ARKV_FMT_E5M2) fp8_encode_kernel<ARKV_FMT_E5M2><<<blocks, 256, 0, s>>>(x, out, n);
+    else fp8_encode_kernel<ARKV_FMT_E4M3><<<blocks, 256, 0, s>>>(x, out, n);
     return cudaGetLastError();
 }
 

@@ -10,8 +10,11 @@ Recipe (one row = one (layer, sequence, kv-head)):
   * prefill keys and values ~ N(0, 1); position 0 is a sink whose key is 4u;
     a share of the other positions are heavy hitters whose key is z + 2u
     (uniform positions, or clustered in non-overlapping spans).
-  * queries (prefill observation queries and decode queries) = z + 0.5u, with u
-    the direction of the query head's kv group.
+  * queries (prefill observation queries and decode queries) = z + a_l u, with u
+    the direction of the query head's kv group and a_l = query_weight(layer), a
+    per-layer weight around 0.5 (0.375 .. 0.625): layers differ in how sharply
+    their attention concentrates on the sink and heavy hitters, so the layers'
+    prefill statistics (and the Original shares drawn from them) differ.
   * decode keys and values appended each step ~ N(0, 1).
   * every value is drawn in float64 and rounded to bfloat16 (via float32, RNE).
 
@@ -28,6 +31,13 @@ from .workloads import Workload
 
 _TENSOR = {"dir": 1, "k": 2, "v": 3, "q_obs": 4, "hh": 5, "q": 6, "k_new": 7,
            "v_new": 8, "ctx": 9}
+
+
+def query_weight(layer: int) -> float:
+    """Weight a_l of the shared direction in layer l's queries: 0.5 + 0.25 (f_l - 0.5)
+    with f_l = frac(0.6180339887 l), an even spread over [0.375, 0.625)."""
+    f = (0.6180339887 * layer) % 1.0
+    return 0.5 + 0.25 * (f - 0.5)
 
 
 def _rng(seed: int, wl: Workload, layer: int, seq: int, head: int, tensor: str,
@@ -108,7 +118,7 @@ def layer_prefill(wl: Workload, layer: int, seed: int = 0, seqs=None, kv_heads=N
             for j in range(G):
                 h = g * G + j
                 z = _rng(seed, wl, layer, b, h, "q_obs").standard_normal((wl.n_obs, D))
-                q_obs[b, h] = round_bf16(z + 0.5 * u)
+                q_obs[b, h] = round_bf16(z + query_weight(layer) * u)
     return {"k": k, "v": v, "q_obs": q_obs, "ctx_len": ctx}
 
 
@@ -124,7 +134,7 @@ def decode_inputs(wl: Workload, layer: int, step: int, seed: int = 0) -> dict:
             for j in range(G):
                 h = g * G + j
                 z = _rng(seed, wl, layer, b, h, "q", step).standard_normal(D)
-                q[b, h] = round_bf16(z + 0.5 * u)
+                q[b, h] = round_bf16(z + query_weight(layer) * u)
             kn[b, g] = round_bf16(_rng(seed, wl, layer, b, g, "k_new", step).standard_normal(D))
             vn[b, g] = round_bf16(_rng(seed, wl, layer, b, g, "v_new", step).standard_normal(D))
     return {"q": q, "k_new": kn, "v_new": vn}
@@ -166,7 +176,7 @@ def layer_prefill_torch(wl: Workload, layer: int, device, seed: int = 0, ctx=Non
                 k[b, g, n:] = 0
                 v[b, g, n:] = 0
     q_obs = torch.randn((B, wl.hq, wl.n_obs, D), generator=gen, device=device, dtype=f32)
-    q_obs += 0.5 * u.repeat_interleave(G, dim=0)[None, :, None, :]
+    q_obs += query_weight(layer) * u.repeat_interleave(G, dim=0)[None, :, None, :]
     bf = torch.bfloat16
     return {"k": k.to(bf), "v": v.to(bf), "q_obs": q_obs.to(bf), "u": u,
             "ctx_len": torch.as_tensor(np.asarray(ctx, np.int32), device=device)}
@@ -184,7 +194,7 @@ def decode_inputs_torch(wl: Workload, u: "torch.Tensor", steps: int, device, see
     gen = torch.Generator(device=device)
     gen.manual_seed((seed * 1000033 + wl.cfg_id * 104729 + layer + 17) & 0x7FFFFFFFFFFF)
     q = torch.randn((steps, B, wl.hq, D), generator=gen, device=device)
-    q += 0.5 * u.repeat_interleave(G, dim=0)[None, None]
+    q += query_weight(layer) * u.repeat_interleave(G, dim=0)[None, None]
     kn = torch.randn((steps, B, Hkv, D), generator=gen, device=device)
     vn = torch.randn((steps, B, Hkv, D), generator=gen, device=device)
     bf = torch.bfloat16

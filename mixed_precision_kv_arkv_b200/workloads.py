@@ -32,6 +32,7 @@ class Workload:
     hh_spans: int = 0         # 0: heavy hitters uniform; else clustered in this many spans
     hh_span_len: int = 512
     r_bar: float = 0.55       # mean Original share when r comes from prefill stats
+    quant_format: str = "e4m3"  # FP8 format of the Quantized tier ("e4m3" or "e5m2")
 
     @property
     def group(self) -> int:
@@ -88,7 +89,9 @@ ALL = (TINY, LLAMA3_3B, LLAMA3_8B, QWEN3_8B, RAGGED)
 LLAMA3_8B_FULL = LLAMA3_8B.with_(name="llama3_8b_full_bf16", budget_frac=1.0, oq_ratio=1.0)
 LLAMA3_8B_BASE_ORIGIN = LLAMA3_8B.with_(name="llama3_8b_base_origin", oq_ratio=1.0)
 LLAMA3_8B_BASE_QUANT = LLAMA3_8B.with_(name="llama3_8b_base_quant", budget_frac=0.52, oq_ratio=0.0)
-MODES = (LLAMA3_8B_FULL, LLAMA3_8B_BASE_ORIGIN, LLAMA3_8B_BASE_QUANT)
+# The same ARKV workload with the Quantized tier in the other FP8 format (E5M2).
+LLAMA3_8B_E5M2 = LLAMA3_8B.with_(name="llama3_8b_e5m2", quant_format="e5m2")
+MODES = (LLAMA3_8B_FULL, LLAMA3_8B_BASE_ORIGIN, LLAMA3_8B_BASE_QUANT, LLAMA3_8B_E5M2)
 
 BY_NAME = {w.name: w for w in ALL + MODES}
 BY_ID = {w.cfg_id: w for w in ALL}

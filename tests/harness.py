@@ -18,18 +18,19 @@ def bits_to_bf16_tensor(bits: np.ndarray, device) -> torch.Tensor:
 
 
 def capacities(wl, r: float, n_max: int):
-    c = make_cfg(wl.batch, wl.hq, wl.hkv, wl.head_dim, wl.window, wl.n_obs, wl.gamma, wl.budget_frac, 1, 1)
+    c = make_cfg(wl.batch, wl.hq, wl.hkv, wl.head_dim, wl.window, wl.n_obs, wl.gamma, wl.budget_frac, 1, 1,
+                 wl.quant_format)
     return abi.arkv_row_capacity(c, n_max, r, wl.reassign_interval)
 
 
 def layer_cfg(wl, cap_o: int, cap_q: int):
     return make_cfg(wl.batch, wl.hq, wl.hkv, wl.head_dim, wl.window, wl.n_obs, wl.gamma,
-                    wl.budget_frac, cap_o, cap_q)
+                    wl.budget_frac, cap_o, cap_q, wl.quant_format)
 
 
 def new_oracle_layer(wl, ctx_len, rows=None) -> A.OracleLayer:
     return A.OracleLayer(wl.batch, wl.hq, wl.hkv, wl.head_dim, wl.window, wl.n_obs, wl.budget_frac,
-                         wl.gamma, ctx_len, rows)
+                         wl.gamma, ctx_len, rows, wl.quant_format)
 
 
 # ------------------------------------------------------------------ oracle -> device

@@ -13,7 +13,7 @@ import torch
 from mixed_precision_kv_arkv_b200 import abi, inputs, workloads
 from mixed_precision_kv_arkv_b200.build import build
 from oracle import arkv as A
-from oracle import e4m3
+from oracle import e4m3, e5m2
 from tests import harness as H
 
 pytestmark = pytest.mark.gpu
@@ -32,8 +32,11 @@ def to_dev(bits, dev):
 
 
 # ------------------------------------------------------------------ FP8 conversion
-def test_fp8_encode_exhaustive(cuda):
-    """All 2^32 float32 bit patterns: device conversion == oracle encoder."""
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+def test_fp8_encode_exhaustive(cuda, fmt):
+    """All 2^32 float32 bit patterns: device conversion == oracle encoder (NaN
+    inputs: a NaN code of the format, sign not compared)."""
+    codec = {"e4m3": e4m3, "e5m2": e5m2}[fmt]
     chunk = 1 << 28
     out = torch.empty(chunk, dtype=torch.uint8, device=cuda)
     idx = torch.arange(chunk, dtype=torch.int64, device=cuda)
@@ -41,13 +44,17 @@ def test_fp8_encode_exhaustive(cuda):
         start = c * chunk
         b = idx + start
         b = torch.where(b >= (1 << 31), b - (1 << 32), b).to(torch.int32).view(torch.float32)
-        abi.arkv_fp8_encode(b.data_ptr(), out.data_ptr(), chunk, H.stream_ptr())
+        abi.arkv_fp8_encode(abi.FORMATS[fmt], b.data_ptr(), out.data_ptr(), chunk, H.stream_ptr())
         got = out.cpu().numpy()
-        ref = e4m3.encode_bits_range(start, chunk)
+        ref = codec.encode_bits_range(start, chunk)
         bits = (np.arange(chunk, dtype=np.uint64) + start).astype(np.uint32)
         isnan = ((bits & 0x7F800000) == 0x7F800000) & ((bits & 0x007FFFFF) != 0)
         assert np.array_equal(got[~isnan], ref[~isnan]), f"chunk {c}"
-        assert ((got[isnan] & 0x7F) == 0x7F).all()
+        g = got[isnan]
+        if fmt == "e4m3":
+            assert ((g & 0x7F) == 0x7F).all()
+        else:   # exponent all ones and a nonzero mantissa
+            assert ((g & 0x7C) == 0x7C).all() and ((g & 0x03) != 0).all()
 
 
 # ------------------------------------------------------------------ scenario runner
@@ -199,7 +206,13 @@ SMALL_D128_G1 = workloads.LLAMA3_3B.with_(name="small_d128_g1", cfg_id=14, layer
 SMALL_D64_G2 = workloads.TINY.with_(name="small_d64_g2", cfg_id=15, hq=4, hkv=2, steps=8)
 
 
-@pytest.mark.parametrize("wl", [SMALL_D128_G3, SMALL_RAGGED, SMALL_CLUSTER, SMALL_D128_G1, SMALL_D64_G2],
+# the Quantization tier in the second FP8 format (E5M2), at both head dims
+SMALL_E5M2_D128 = SMALL_D128_G3.with_(name="small_e5m2_d128", cfg_id=16, quant_format="e5m2")
+TINY_E5M2 = workloads.TINY.with_(name="tiny_e5m2", cfg_id=17, quant_format="e5m2")
+
+
+@pytest.mark.parametrize("wl", [SMALL_D128_G3, SMALL_RAGGED, SMALL_CLUSTER, SMALL_D128_G1, SMALL_D64_G2,
+                                SMALL_E5M2_D128, TINY_E5M2],
                          ids=lambda w: w.name)
 def test_small_workloads(cuda, wl):
     s = run_scenario(wl, wl.steps, cuda)
