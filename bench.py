@@ -5,7 +5,9 @@
 
 A step is one decode step of the whole attention stack: for every layer, append +
 mixed-precision attention (arkv_decode_attn), score update (arkv_score_update),
-and the tier reassignment (arkv_reassign) on every reassign_interval-th step.
+and the tier reassignment (arkv_reassign) on every reassign_interval-th step.  The
+score update and reassignment of a layer run on a second stream, beside the next
+layers' attention; the layer's next attention call waits for them.
 Each GPU runs its own replica of the workload (independent sequences; no
 collective on the data path), so `value` is the tokens/s of all ranks together
 ("scaling": "weak").  Inputs are synthetic and seeded; each step streams the whole
@@ -235,7 +237,8 @@ def cpu_baseline_from_state(wl, lay0, ctx_np, t_next, o_dev, seconds, decode_ste
 
     # the step both sides take from the same state
     decode_step_dev(t_next)
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
     t0 = time.perf_counter()
     o_ref = oracle_step(t_next)
     first = time.perf_counter() - t0
@@ -387,28 +390,52 @@ def run_arkv(args, wl, rank, world, local_rank):
     o = torch.zeros((L, B, Hq, D), dtype=torch.float32, device=dev)
     launches = {"n": 0}
 
+    # The score update and reassignment of layer l run on a side stream: the next
+    # layer's attention does not wait for them (in a model, the next layer's query
+    # needs only this layer's output).  The next call on layer l's cache waits for them.
+    side = torch.cuda.Stream(device=dev)
+    pending = {}                                             # layer -> event after its side work
+
+    def settle(l):
+        ev_done = pending.pop(l, None)
+        if ev_done is not None:
+            torch.cuda.current_stream().wait_event(ev_done)
+
+    def join():
+        for l in list(pending):
+            settle(l)
+
     def layer_step(l, t, q=None, kn=None, vn=None, ev=None):
         x = layers[l]
         cfg, c = x["cfg"], x["cache"].c
         q = x["dec"]["q"][t] if q is None else q
         kn = x["dec"]["k_new"][t] if kn is None else kn
         vn = x["dec"]["v_new"][t] if vn is None else vn
+        settle(l)
+        main = torch.cuda.current_stream()
         if ev is not None:
-            ev[0].record()
+            ev[0].record(main)
         abi.arkv_decode_attn(cfg, t, q.data_ptr(), kn.data_ptr(), vn.data_ptr(), ctx.data_ptr(), c,
-                             o[l].data_ptr(), x["ws_d"].ptr, x["ws_d"].nbytes, stream_ptr())
+                             o[l].data_ptr(), x["ws_d"].ptr, x["ws_d"].nbytes, main.cuda_stream)
         if ev is not None:
-            ev[1].record()
-        abi.arkv_score_update(cfg, t, ctx.data_ptr(), c, x["ws_d"].ptr, x["ws_d"].nbytes, stream_ptr())
+            ev[1].record(main)
+        attended = torch.cuda.Event()
+        attended.record(main)
+        side.wait_event(attended)
+        abi.arkv_score_update(cfg, t, ctx.data_ptr(), c, x["ws_d"].ptr, x["ws_d"].nbytes, side.cuda_stream)
         launches["n"] += KERNELS_PER_LAYER_STEP
         if (t + 1) % wl.reassign_interval == 0:
             abi.arkv_reassign(cfg, t, x["r"], ctx.data_ptr(), c, None, x["ws_r"].ptr, x["ws_r"].nbytes,
-                              stream_ptr())
+                              side.cuda_stream)
             launches["n"] += 1
+        done = torch.cuda.Event()
+        done.record(side)
+        pending[l] = done
 
     for t in range(W):                                       # warm-up, eager
         for l in range(L):
             layer_step(l, t)
+    join()
     torch.cuda.synchronize()
 
     def capture(t0, nsteps, body):
@@ -419,6 +446,7 @@ def run_arkv(args, wl, rank, world, local_rank):
             with torch.cuda.graph(g):
                 for tt in range(t, t + n):
                     body(tt)
+                join()                                       # the side stream rejoins the capture
             graphs.append(g)
             t += n
         return graphs
@@ -464,6 +492,7 @@ def run_arkv(args, wl, rank, world, local_rank):
     def k_body(tt):
         i = tt - t_k
         for l in range(L):
+            settle(l)
             counts[i, l, 0].copy_(layers[l]["cache"].n_bf16)
             counts[i, l, 1].copy_(layers[l]["cache"].n_fp8)
             layer_step(l, tt, ev=evs[i * L + l])
@@ -521,7 +550,7 @@ def run_arkv(args, wl, rank, world, local_rank):
                        "ms_per_step": ms_e2e / K}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_from_state(wl, layers[0], ctx_np, total_steps, o, args.cpu_seconds,
-                                                       lambda t: layer_step(0, t))
+                                                       lambda t: (layer_step(0, t), join()))
     if rank == 0:
         print(json.dumps(line), flush=True)
     del g_value, g_k

@@ -92,6 +92,12 @@ def test_null_cache_buffers_and_small_workspace_rejected(lib):
                                 check=False) == abi.ARKV_EINVAL
     assert abi.arkv_reassign(c, 0, 1.5, p, cache, None, p, 1 << 30, None,
                              check=False) == abi.ARKV_EINVAL
+    # the attention output is written in 16-byte words
+    assert abi.arkv_decode_attn(c, 0, p, p, p, p, cache, p + 4, p, need, None,
+                                check=False) == abi.ARKV_EINVAL
+    assert "aligned" in abi.arkv_last_error_string()
+    # unknown FP8 format of the debug encoder
+    assert abi.arkv_fp8_encode(7, p, p, 16, None, check=False) == abi.ARKV_EINVAL
     # capacities below the kept counts at the longest context are refused up front
     small = cfg(cap_bf16=10, cap_fp8=10)
     assert abi.arkv_quantize_pack(small, 0.5, p, p, 2048, p, p, p, cache, None, p, 1 << 30, None,
