@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--streams", type=int, default=2, choices=[1, 2],
+                    help="2: score updates and reassignments on a second stream beside the next layers' "
+                         "attention; 1: everything on one stream")
     ap.add_argument("--layers", type=int, default=None,
                     help="run only this many layers of the workload (profiling a smaller case)")
     return ap.parse_args()
@@ -314,12 +317,13 @@ def run_reference(args, wl, rank):
     print(json.dumps(line), flush=True)
 
 
-def config_of(wl):
+def config_of(wl, streams=2):
     return {"workload": wl.name, "layers": wl.layers, "batch": wl.batch, "hq": wl.hq, "hkv": wl.hkv,
             "head_dim": wl.head_dim, "n_ctx": wl.n_ctx, "n_ctx_min": wl.n_ctx_min,
             "budget_frac": wl.budget_frac, "oq_ratio": wl.oq_ratio if wl.oq_ratio is not None
             else f"per layer from prefill stats (r_bar {wl.r_bar})", "window": wl.window,
             "gamma": wl.gamma, "reassign_interval": wl.reassign_interval, "quant_format": wl.quant_format,
+            "streams": "score update and reassignment on a second stream" if streams == 2 else "one stream",
             "l2": "no flush: every step streams the whole compressed cache, far above L2"}
 
 
@@ -393,7 +397,7 @@ def run_arkv(args, wl, rank, world, local_rank):
     # The score update and reassignment of layer l run on a side stream: the next
     # layer's attention does not wait for them (in a model, the next layer's query
     # needs only this layer's output).  The next call on layer l's cache waits for them.
-    side = torch.cuda.Stream(device=dev)
+    side = torch.cuda.Stream(device=dev) if args.streams == 2 else None
     pending = {}                                             # layer -> event after its side work
 
     def settle(l):
@@ -419,18 +423,21 @@ def run_arkv(args, wl, rank, world, local_rank):
                              o[l].data_ptr(), x["ws_d"].ptr, x["ws_d"].nbytes, main.cuda_stream)
         if ev is not None:
             ev[1].record(main)
-        attended = torch.cuda.Event()
-        attended.record(main)
-        side.wait_event(attended)
-        abi.arkv_score_update(cfg, t, ctx.data_ptr(), c, x["ws_d"].ptr, x["ws_d"].nbytes, side.cuda_stream)
+        aux = side if side is not None else main
+        if side is not None:
+            attended = torch.cuda.Event()
+            attended.record(main)
+            side.wait_event(attended)
+        abi.arkv_score_update(cfg, t, ctx.data_ptr(), c, x["ws_d"].ptr, x["ws_d"].nbytes, aux.cuda_stream)
         launches["n"] += KERNELS_PER_LAYER_STEP
         if (t + 1) % wl.reassign_interval == 0:
             abi.arkv_reassign(cfg, t, x["r"], ctx.data_ptr(), c, None, x["ws_r"].ptr, x["ws_r"].nbytes,
-                              side.cuda_stream)
+                              aux.cuda_stream)
             launches["n"] += 1
-        done = torch.cuda.Event()
-        done.record(side)
-        pending[l] = done
+        if side is not None:
+            done = torch.cuda.Event()
+            done.record(side)
+            pending[l] = done
 
     for t in range(W):                                       # warm-up, eager
         for l in range(L):
@@ -530,7 +537,7 @@ def run_arkv(args, wl, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": ms_value / K, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_of(wl),
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_of(wl, args.streams),
         "hbm_gbs_step": step_bytes / (ms_value / K * 1e-3) / 1e9,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": kernel_traffic("decode_attn.cu"),

@@ -122,7 +122,9 @@ struct LayerDims {
 
 struct AttnParams {
     CUtensorMap tm_k16, tm_v16;   // [R*cap_bf16][D] bf16, boxes of 16 rows x 128 bytes, 128B swizzle
-    CUtensorMap tm_k8, tm_v8;     // [R*cap_fp8][D] E4M3, boxes of 16 rows x min(D,128) bytes
+    CUtensorMap tm_k8, tm_v8;     // [R*cap_fp8][D] FP8 codes, boxes of 16 rows x D bytes
+    CUtensorMap tm_k16b, tm_v16b; // the same arrays, boxes of one ring stage's rows
+    CUtensorMap tm_k8b, tm_v8b;
     LayerDims d;
     int step;
     const uint16_t* q;

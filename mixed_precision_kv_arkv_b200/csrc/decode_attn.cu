@@ -3,9 +3,8 @@
 // originals) and the score observation that feeds §2.나.
 //
 // One wave of CTAs (as many as the GPU holds at once) shares the rows in
-// proportion to their lengths; each CTA takes an equal share of its row, counted
-// in 16-token tiles (a bf16 tile weighs two FP8 tiles, its bytes), bf16 tiles first
-// and FP8 tiles after.  Its 4 warps take the tiles round robin, each through its
+// proportion to their lengths; each CTA takes the same fraction of its row's bf16
+// tiles and of its FP8 tiles (16 tokens each), bf16 tiles first.  Its 4 warps take the tiles round robin, each through its
 // own ring of 4 shared-memory slots (a bf16 tile takes two, K then V; an FP8 tile
 // one) filled by TMA tensor loads (16 rows per box, 128-byte swizzle; 64-byte for
 // FP8 rows of 64 bytes) completing on per-slot mbarriers (waits are bounded).
@@ -63,6 +62,7 @@ constexpr int kWarps = 4;
 constexpr int kSlots = 4;                  // ring slots per warp: a bf16 tile takes 2, an FP8 tile 1
 constexpr int kSpinLimit = 1 << 20;        // bounded mbarrier waits (~1 s worst case)
 constexpr int kMaxGrid = 2048;             // CTAs of one call at most (partial slots in the workspace)
+constexpr int kScaleTokens = 512;          // FP8 scales a CTA keeps in shared memory (the rest from L2)
 
 // ------------------------------------------------------------------ shared-memory layout
 template <int D>
@@ -76,7 +76,9 @@ struct Smem {
     static constexpr int kMax = kRed + 16 * 4;                          // float [4]
     static constexpr int kAbort = kMax + 16;                            // int: a wait gave up
     static constexpr int kShare = kAbort + 16;                          // int [4]: row, index, count, base
-    static constexpr int kBytes = kShare + 16 + 1024;                   // + alignment slack
+    static constexpr int kScales = kShare + 16;                         // float [2][kScaleTokens]: sk, sv
+    static constexpr int kVmax = kScales + 2 * kScaleTokens * 4;        // float [4]
+    static constexpr int kBytes = kVmax + 16 + 1024;                    // + alignment slack
     static constexpr int kO = 0;                                        // float [4][4][D], in the idle ring
     static_assert(4 * 4 * D * 4 <= kRing, "the epilogue buffer must fit in the ring");
 };
@@ -560,17 +562,30 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
 #pragma unroll
     for (int mt = 0; mt < KB; ++mt) oacc[mt][0] = oacc[mt][1] = oacc[mt][2] = oacc[mt][3] = 0.f;
 
-    // the largest V scale of the warp's FP8 tiles (1 if it has none); every tile's P is
-    // multiplied by vnorm = 64 / vmax (p < 2^8: p sv vnorm < 2^14, inside f16)
+    // the CTA's FP8 scales: the first kScaleTokens into shared memory, one coalesced
+    // pass by the whole CTA that also finds the largest V scale (64 if there is none);
+    // every tile's P is multiplied by vnorm = 64 / vmax (p < 2^8: p sv vnorm < 2^14,
+    // inside f16)
     const float* skb = p.c.sk + (size_t)row * d.cap_q;
     const float* svb = p.c.sv + (size_t)row * d.cap_q;
-    float vmax = 0.f;
-    for (int i = nt16; i < nt; ++i) {
-        const int tk = 16 * tile_of(i) + (lane & 15);
-        if (tk < n8) vmax = fmaxf(vmax, __ldg(svb + tk));
+    float* sm_sk = reinterpret_cast<float*>(smem + SL::kScales);
+    float* sm_sv = sm_sk + kScaleTokens;
+    float* sm_vmax = reinterpret_cast<float*>(smem + SL::kVmax);
+    const int tq0 = 16 * a8, tq1 = min(16 * e8, n8);
+    float vm = 0.f;
+    for (int k = tq0 + tid; k < tq1; k += blockDim.x) {
+        const float v = __ldg(svb + k);
+        vm = fmaxf(vm, v);
+        if (k - tq0 < kScaleTokens) {
+            sm_sk[k - tq0] = __ldg(skb + k);
+            sm_sv[k - tq0] = v;
+        }
     }
 #pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(kFull, vmax, m));
+    for (int m = 16; m >= 1; m >>= 1) vm = fmaxf(vm, __shfl_xor_sync(kFull, vm, m));
+    if (lane == 0) sm_vmax[warp] = vm;
+    __syncthreads();
+    float vmax = fmaxf(fmaxf(sm_vmax[0], sm_vmax[1]), fmaxf(sm_vmax[2], sm_vmax[3]));
     if (!(vmax > 0.f)) vmax = 64.f;
     const float vnorm = 64.f / vmax;
 
@@ -622,25 +637,24 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
         const LaneOffsets<D, true> off;
         float* logit_head = p.logit8 + ((size_t)row * 4 + (hv ? hd : 0)) * p.lstride_q;
         const int s1 = min(n8, e8 * 16);
-        float nsk[4], nsv[4];
-        auto load_scales = [&](int t0) {
+        for (int i = nt16; i < nt; ++i) {
+            const int t0 = 16 * tile_of(i);
+            float skv[4], svv[4];
             const int tok[4] = {t0 + 2 * t, t0 + 2 * t + 1, t0 + 8 + 2 * t, t0 + 9 + 2 * t};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int k = min(tok[e], d.cap_q - 1);
-                nsk[e] = __ldg(skb + k);
-                nsv[e] = __ldg(svb + k);
+                const int k = tok[e] - tq0;
+                if (k < kScaleTokens) {               // tokens past the segment end get stale values
+                    skv[e] = sm_sk[min(k, kScaleTokens - 1)];
+                    svv[e] = sm_sv[min(k, kScaleTokens - 1)];
+                } else {
+                    skv[e] = __ldg(skb + min(tok[e], d.cap_q - 1));
+                    svv[e] = __ldg(svb + min(tok[e], d.cap_q - 1));
+                }
             }
-        };
-        load_scales(16 * tile_of(nt16));
-        for (int i = nt16; i < nt; ++i) {
             if (!wait_tile(i)) { aborted = true; break; }
-            float skv[4], svv[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) { skv[e] = nsk[e]; svv[e] = nsv[e]; }
-            if (i + 1 < nt) load_scales(16 * tile_of(i + 1));
-            attend_tile<D, true, FMT>(ring + pos * SLOT, off, 16 * tile_of(i), s1, hv, lo, c2, skv, svv, vnorm,
-                                      logit_head, qa, rs, oacc);
+            attend_tile<D, true, FMT>(ring + pos * SLOT, off, t0, s1, hv, lo, c2, skv, svv, vnorm, logit_head, qa,
+                                      rs, oacc);
             release(1);
         }
     }
@@ -784,13 +798,11 @@ __global__ void __launch_bounds__(32 * kWarps, ARKV_MIN_CTAS) decode_attn_kernel
     const int n8 = min(max(p.c.n_fp8[row], 0), d.cap_q);          // capacities before any use
     const bool append = n16_old < d.cap_o;
     const int n16 = n16_old + (append ? 1 : 0);                    // the new token included
-    // this CTA's share of the row, in units of 16-token FP8 tiles (a bf16 tile counts
-    // two): tile j of bf16 starts at unit 2j, FP8 tile j at 2 T16 + j; the CTA takes
-    // the tiles starting in [u0, u1)
-    const int T16 = (n16 + 15) / 16, T8 = (n8 + 15) / 16, U = 2 * T16 + T8;
-    const int u0 = (int)((long long)U * sh.c / sh.n), u1 = (int)((long long)U * (sh.c + 1) / sh.n);
-    const int a16 = min((u0 + 1) / 2, T16), e16 = min((u1 + 1) / 2, T16);
-    const int a8 = min(max(u0 - 2 * T16, 0), T8), e8 = min(max(u1 - 2 * T16, 0), T8);
+    // this CTA's share of the row: the same fraction of each segment's 16-token tiles,
+    // so that every CTA of the row has the same mix of bf16 and FP8 work
+    const int T16 = (n16 + 15) / 16, T8 = (n8 + 15) / 16;
+    const int a16 = (int)((long long)T16 * sh.c / sh.n), e16 = (int)((long long)T16 * (sh.c + 1) / sh.n);
+    const int a8 = (int)((long long)T8 * sh.c / sh.n), e8 = (int)((long long)T8 * (sh.c + 1) / sh.n);
 
     if (e16 > a16 || e8 > a8) {
         if (lane == 0) {
