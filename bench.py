@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--streams", type=int, default=2, choices=[1, 2],
                     help="2: score updates and reassignments on a second stream beside the next layers' "
                          "attention; 1: everything on one stream")
+    ap.add_argument("--no-early-start", action="store_true",
+                    help="launch every attention call with early_start = 0 (it waits for the previous "
+                         "kernel before reading its cache)")
     ap.add_argument("--layers", type=int, default=None,
                     help="run only this many layers of the workload (profiling a smaller case)")
     return ap.parse_args()
@@ -317,14 +320,15 @@ def run_reference(args, wl, rank):
     print(json.dumps(line), flush=True)
 
 
-def config_of(wl, streams=2):
+def config_of(wl, streams=2, early=None):
     return {"workload": wl.name, "layers": wl.layers, "batch": wl.batch, "hq": wl.hq, "hkv": wl.hkv,
             "head_dim": wl.head_dim, "n_ctx": wl.n_ctx, "n_ctx_min": wl.n_ctx_min,
             "budget_frac": wl.budget_frac, "oq_ratio": wl.oq_ratio if wl.oq_ratio is not None
             else f"per layer from prefill stats (r_bar {wl.r_bar})", "window": wl.window,
             "gamma": wl.gamma, "reassign_interval": wl.reassign_interval, "quant_format": wl.quant_format,
             "streams": "score update and reassignment on a second stream" if streams == 2 else "one stream",
-            "l2": "no flush: every step streams the whole compressed cache, far above L2"}
+            "l2": "no flush: every step streams the whole compressed cache, far above L2",
+            "early_start": (wl.layers >= 3) if early is None else bool(early)}
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -342,7 +346,7 @@ def run_arkv(args, wl, rank, world, local_rank):
     s = stream_ptr()
     L, B, Hq, Hkv, D = wl.layers, wl.batch, wl.hq, wl.hkv, wl.head_dim
     K, W = args.steps, args.warmup
-    passes = 1 + (0 if args.no_e2e else 1) + 1          # value, e2e, kernel timing
+    passes = 1 + (0 if args.no_e2e else 1) + 1          # value, e2e, per-call kernel timing
     total_steps = W + passes * K
     ctx_np = inputs.ctx_lengths(wl, 0)
     n_max = int(ctx_np.max()) + total_steps + 1        # + the step the CPU baseline checks
@@ -350,6 +354,9 @@ def run_arkv(args, wl, rank, world, local_rank):
 
     # ---------- prefill statistics of every layer, then the per-layer Original share
     probe = make_cfg(B, Hq, Hkv, D, wl.window, wl.n_obs, wl.gamma, wl.budget_frac, 1, 1, wl.quant_format)
+    # consecutive attention calls on the main stream belong to different layers, so with
+    # three or more layers each may read its cache before the previous kernel ends
+    early = L >= 3 and not args.no_early_start
     ws_pre = Workspace(abi.arkv_workspace_bytes(probe, abi.ARKV_WS_PREFILL, wl.n_ctx), dev)
     stats = torch.zeros((L, 3), dtype=torch.float64, device=dev)
     mu0 = torch.zeros((wl.rows, wl.n_ctx), dtype=torch.float64, device=dev)
@@ -371,9 +378,11 @@ def run_arkv(args, wl, rank, world, local_rank):
     # ---------- per-layer caches: capacities, initial pack
     layers = []
     for l in range(L):
-        cap_o, cap_q = abi.arkv_row_capacity(probe, n_max, float(r[l]), wl.reassign_interval)
+        # K slots beyond the workload's need: the pipelined kernel pass appends K tokens
+        # with no reassignment between (its appends are rolled back afterwards)
+        cap_o, cap_q = abi.arkv_row_capacity(probe, n_max, float(r[l]), wl.reassign_interval + K)
         cfg = make_cfg(B, Hq, Hkv, D, wl.window, wl.n_obs, wl.gamma, wl.budget_frac, cap_o, cap_q,
-                       wl.quant_format)
+                       wl.quant_format, early_start=early)
         cache = LayerCache(cfg, dev)
         pre = inputs.layer_prefill_torch(wl, l, dev, seed, ctx_np)
         abi.arkv_prefill_stats(cfg, pre["q_obs"].data_ptr(), pre["k"].data_ptr(), wl.n_ctx,
@@ -505,6 +514,18 @@ def run_arkv(args, wl, rank, world, local_rank):
             layer_step(l, tt, ev=evs[i * L + l])
     g_k = capture(t_k, K, k_body)
 
+    # ---------- pass 4: the attention calls alone, K steps of L back-to-back launches on
+    # one stream (each may overlap the tail of the one before it), timed as a whole;
+    # replayed on the state pass 3 leaves, and rolled back afterwards (n_bf16 restored)
+    def pipe_body(tt):
+        for l in range(L):
+            x = layers[l]
+            abi.arkv_decode_attn(x["cfg"], tt, x["dec"]["q"][tt].data_ptr(), x["dec"]["k_new"][tt].data_ptr(),
+                                 x["dec"]["v_new"][tt].data_ptr(), ctx.data_ptr(), x["cache"].c,
+                                 o[l].data_ptr(), x["ws_d"].ptr, x["ws_d"].nbytes,
+                                 torch.cuda.current_stream().cuda_stream)
+    g_pipe = capture(t_k, K, pipe_body)
+
     def timed(graphs):
         if world > 1:
             dist.barrier()
@@ -521,14 +542,31 @@ def run_arkv(args, wl, rank, world, local_rank):
         ms_value = timed(g_value)
         ms_e2e = timed(g_e2e) if not args.no_e2e else None
         timed(g_k)
+        join()
+        saved = [(x["cache"].n_bf16.clone(), x["cache"].n_fp8.clone()) for x in layers]
+        torch.cuda.synchronize()
+        ms_pipe = timed(g_pipe)
+        for x, (n16, n8) in zip(layers, saved):
+            x["cache"].n_bf16.copy_(n16)
+    torch.cuda.synchronize()
+    outputs_finite = bool(torch.isfinite(o).all())            # every layer's output of the last step
     clocks = clk.summary()
-    clocks["window"] = "sampled every 50 ms across the three timed passes"
+    clocks["window"] = "sampled every 50 ms across the four timed passes"
+    io_bytes = B * Hq * D * 2 + B * Hq * D * 4 + 2 * B * Hkv * D * 2
+    # per-call timing (pass 3): events around each launch inside the full step
     k1_ms = [a.elapsed_time(b) for a, b in evs]
     cn = counts.cpu().numpy().astype(np.int64)               # [K, L, 2, rows] before each launch
     per_row = (cn[:, :, 0] + 1) * 4 * D + cn[:, :, 1] * (2 * D + 8)
-    io_bytes = B * Hq * D * 2 + B * Hq * D * 4 + 2 * B * Hkv * D * 2
     alg_bytes = per_row.sum(-1) + io_bytes                   # [K, L]
-    achieved = float(alg_bytes.sum() / (sum(k1_ms) * 1e-3) / 1e9)
+    achieved_iso = float(alg_bytes.sum() / (sum(k1_ms) * 1e-3) / 1e9)
+    # pipelined timing (pass 4): launch i of layer l sees n_bf16 = saved + i
+    n16_0 = np.stack([n16.cpu().numpy() for n16, _ in saved]).astype(np.int64)      # [L, rows]
+    n8_0 = np.stack([n8.cpu().numpy() for _, n8 in saved]).astype(np.int64)
+    steps_i = np.arange(K, dtype=np.int64)[:, None, None]
+    pipe_row = (n16_0[None] + steps_i + 1) * 4 * D + n8_0[None] * (2 * D + 8)       # [K, L, rows]
+    pipe_bytes = pipe_row.sum(-1) + io_bytes
+    ms_per_pipe = ms_pipe / (K * L)
+    achieved = float(pipe_bytes.sum() / (ms_pipe * 1e-3) / 1e9)
     peak, peak_kind = hbm_peak()
     step_bytes = float(alg_bytes.sum(-1).mean())
 
@@ -537,19 +575,27 @@ def run_arkv(args, wl, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": ms_value / K, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_of(wl, args.streams),
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_of(wl, args.streams, early),
         "hbm_gbs_step": step_bytes / (ms_value / K * 1e-3) / 1e9,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": kernel_traffic("decode_attn.cu"),
                      "kernel": f"arkv_decode_attn call: decode_attn_kernel<{D}> (split merge fused)",
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                      else "fallback 6650 GB/s",
-                     "bytes_per_launch": float(alg_bytes.mean()),
-                     "ms_per_launch": statistics.mean(k1_ms)},
+                     "timing": f"CUDA events around {K} x {L} back-to-back launches on one stream "
+                               f"(early_start={int(early)}), per-launch mean",
+                     "bytes_per_launch": float(pipe_bytes.mean()),
+                     "ms_per_launch": ms_per_pipe,
+                     "isolated": {"timing": "CUDA events around each launch inside the full step "
+                                            "(score updates on the side stream running beside it)",
+                                  "achieved": achieved_iso, "frac": achieved_iso / peak,
+                                  "bytes_per_launch": float(alg_bytes.mean()),
+                                  "ms_per_launch": statistics.mean(k1_ms)}},
         "gpu_launches": gpu_launches,
         "clocks": clocks,
         "oq_ratio_per_layer": [round(float(x), 4) for x in r],
         "cache_status": status,
+        "outputs_finite": outputs_finite,
     }
     if not args.no_e2e:
         line["e2e"] = {"value": job_tokens_per_s(B, K, world, ms_e2e), "unit": "tokens/s",
@@ -560,7 +606,7 @@ def run_arkv(args, wl, rank, world, local_rank):
                                                        lambda t: (layer_step(0, t), join()))
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del g_value, g_k
+    del g_value, g_k, g_pipe
     if not args.no_e2e:
         del g_e2e
 

@@ -89,6 +89,7 @@ typedef struct arkv_cfg {
     int32_t cap_bf16;       /* slots per row, bf16 segment */
     int32_t cap_fp8;        /* slots per row, fp8 segment */
     int32_t quant_format;   /* ARKV_FMT_*: FP8 format of the Quantized tier */
+    int32_t early_start;    /* 0 or 1, arkv_decode_attn only: see there */
 } arkv_cfg;
 
 /* Device buffers of one layer's packed cache (see Layout above). */
@@ -176,7 +177,16 @@ int arkv_quantize_pack(const arkv_cfg *cfg, float r, const uint16_t *k, const ui
  *   all four 16-byte aligned.
  * The row's bf16 count (n_bf16) is advanced past the new token when the call
  * completes.  A full bf16 segment sets ARKV_STATUS_BF16_FULL and drops the new
- * token. */
+ * token.
+ * The kernel is launched as a programmatic dependent of the kernel before it on
+ * the stream, and lets the kernel after it launch the same way: its blocks may be
+ * resident before the previous kernel has finished.  With cfg->early_start = 0
+ * they read nothing before it has finished and its writes are visible.  With
+ * cfg->early_start = 1 they first read this layer's cache (codes, scales, counts
+ * n_bf16 and n_fp8) and ctx_len, and wait only before q, k_new, v_new, o, ws and
+ * every write: set it only when neither of the two kernels that precede the call
+ * on the stream writes those buffers (for example, consecutive calls on other
+ * layers' caches). */
 int arkv_decode_attn(const arkv_cfg *cfg, int32_t step, const uint16_t *q, const uint16_t *k_new,
                      const uint16_t *v_new, const int32_t *ctx_len, arkv_layer_cache *cache,
                      float *o, void *ws, size_t ws_bytes, arkv_stream_t stream);

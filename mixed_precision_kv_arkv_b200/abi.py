@@ -26,7 +26,8 @@ class arkv_cfg(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("window", ctypes.c_int32), ("n_obs", ctypes.c_int32),
                 ("gamma", ctypes.c_float), ("budget_frac", ctypes.c_float),
                 ("cap_bf16", ctypes.c_int32), ("cap_fp8", ctypes.c_int32),
-                ("quant_format", ctypes.c_int32)]
+                ("quant_format", ctypes.c_int32),
+                ("early_start", ctypes.c_int32)]
 
 
 class arkv_layer_cache(ctypes.Structure):

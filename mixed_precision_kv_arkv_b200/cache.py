@@ -12,9 +12,9 @@ from . import abi
 
 
 def make_cfg(batch, hq, hkv, head_dim, window, n_obs, gamma, budget_frac, cap_bf16, cap_fp8,
-             quant_format="e4m3"):
+             quant_format="e4m3", early_start=False):
     return abi.arkv_cfg(batch, hq, hkv, head_dim, window, n_obs, float(gamma), float(budget_frac),
-                        cap_bf16, cap_fp8, abi.FORMATS[quant_format])
+                        cap_bf16, cap_fp8, abi.FORMATS[quant_format], int(bool(early_start)))
 
 
 class LayerCache:

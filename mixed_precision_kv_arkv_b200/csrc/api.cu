@@ -39,6 +39,7 @@ int check_cfg(const arkv_cfg* c) {
     if (c->cap_bf16 < 1 || c->cap_fp8 < 1) return fail(ARKV_EINVAL, "%s: capacities must be >= 1", "cfg");
     if (c->quant_format != ARKV_FMT_E4M3 && c->quant_format != ARKV_FMT_E5M2)
         return fail(ARKV_EINVAL, "%s: quant_format must be ARKV_FMT_E4M3 or ARKV_FMT_E5M2", "cfg");
+    if (c->early_start != 0 && c->early_start != 1) return fail(ARKV_EINVAL, "%s: early_start must be 0 or 1", "cfg");
     return ARKV_OK;
 }
 
@@ -203,6 +204,7 @@ int arkv_decode_attn(const arkv_cfg* cfg, int32_t step, const uint16_t* q, const
     p.lstride_o = w.lstride_o;
     p.lstride_q = w.lstride_q;
     p.inv_sqrt_d = 1.0 / sqrt((double)d.D);
+    p.early_start = cfg->early_start;
     const cudaError_t e = arkv::launch_decode_attn(p, (cudaStream_t)stream);   // also encodes the tensor maps
     return e == cudaSuccess ? ARKV_OK : cuda_fail(e, "arkv_decode_attn");
 }

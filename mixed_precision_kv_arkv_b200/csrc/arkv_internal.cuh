@@ -123,8 +123,6 @@ struct LayerDims {
 struct AttnParams {
     CUtensorMap tm_k16, tm_v16;   // [R*cap_bf16][D] bf16, boxes of 16 rows x 128 bytes, 128B swizzle
     CUtensorMap tm_k8, tm_v8;     // [R*cap_fp8][D] FP8 codes, boxes of 16 rows x D bytes
-    CUtensorMap tm_k16b, tm_v16b; // the same arrays, boxes of one ring stage's rows
-    CUtensorMap tm_k8b, tm_v8b;
     LayerDims d;
     int step;
     const uint16_t* q;
@@ -141,6 +139,7 @@ struct AttnParams {
     unsigned* counter;  // [R]  the rows' tickets (zero between calls)
     int lstride_o, lstride_q;
     double inv_sqrt_d;
+    int early_start;    // read the cache before waiting for the previous kernel
 };
 
 struct ScoreParams {

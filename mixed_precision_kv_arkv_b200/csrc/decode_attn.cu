@@ -75,8 +75,8 @@ struct Smem {
     static constexpr int kRed = kL + 16 * 4;                            // float [4][4]
     static constexpr int kMax = kRed + 16 * 4;                          // float [4]
     static constexpr int kAbort = kMax + 16;                            // int: a wait gave up
-    static constexpr int kShare = kAbort + 16;                          // int [4]: row, index, count, base
-    static constexpr int kScales = kShare + 16;                         // float [2][kScaleTokens]: sk, sv
+    static constexpr int kShare = kAbort + 16;                          // int [8] + int64 [4]: grid share
+    static constexpr int kScales = kShare + 64;                         // float [2][kScaleTokens]: sk, sv
     static constexpr int kVmax = kScales + 2 * kScaleTokens * 4;        // float [4]
     static constexpr int kBytes = kVmax + 16 + 1024;                    // + alignment slack
     static constexpr int kO = 0;                                        // float [4][4][D], in the idle ring
@@ -151,6 +151,16 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     for (int i = 0; i < kSpinLimit; ++i)
         if (mbar_try_wait(bar, parity)) return true;
     return false;
+}
+
+// Programmatic dependent launch: let the next kernel on the stream launch (its
+// blocks take SM slots as this grid's blocks exit), and wait until the kernel
+// before this one has finished with its writes visible.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void prefetch_map(const CUtensorMap* m) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
 // d += a * b on m16n8k16 (f16 or bf16 operands, float32 accumulate).
@@ -451,62 +461,91 @@ __device__ __forceinline__ void load_q(const AttnParams& p, int row, bool fp8, u
 
 // This CTA's place in the grid: the call runs one wave of P CTAs, shared among the
 // rows in proportion to their lengths.  Row r gets n_r = base(r+1) - base(r) >= 1
-// CTAs, base(r) = r + floor((P - R) Wb(r) / Wtot + 1/2) with Wb(r) the summed
-// lengths (ctx_len of the row's sequence + step + 1) of the rows before it.  Only
-// ctx_len enters, which no CTA modifies, so every CTA derives the same shares.
+// CTAs, base(r) = r + F(Wb(r)), F(w) = floor((2 (P - R) w + Wtot) / (2 Wtot)) (the
+// nearest integer to w (P - R) / Wtot, exact), with Wb(r) the summed lengths
+// (ctx_len of the row's sequence + step + 1) of the rows before it.  F is monotone
+// with F(0) = 0 and F(Wtot) = P - R; it is exact integer arithmetic on ctx_len
+// (which no CTA modifies), so every CTA, and every thread that meets a boundary
+// from either side, derives the same shares -- a floating-point F would not: equal
+// lengths put w (P - R) / Wtot + 1/2 exactly on integers, where two evaluations of
+// the same formula may round apart.  The CTA's 128 threads own
+// contiguous runs of rows: one block scan gives Wb, and the thread whose run holds
+// this CTA's row also hands over that row's counts, loaded with the lengths.
 struct Share {
-    int row, c, n, base;
+    int row, c, n, base, n16, n8;
 };
 
-__device__ __forceinline__ Share grid_share(const AttnParams& p, int* sm) {
+__device__ __forceinline__ Share grid_share(const AttnParams& p, char* sm) {
+    constexpr int kRowsReg = 4;   // rows per thread whose counts are loaded up front
     const LayerDims& d = p.d;
-    const int lane = threadIdx.x & 31, bid = blockIdx.x, P = gridDim.x;
-    if (threadIdx.x < 32) {
-        const long long extra = P - d.R;   // CTAs beyond one per row
-        long long tot = 0;
-        for (int b0 = 0; b0 < d.batch; b0 += 32) {
-            const int b = b0 + lane;
-            long long L = b < d.batch ? (long long)__ldg(&p.ctx_len[b]) + p.step + 1 : 0;
+    int* out = reinterpret_cast<int*>(sm);
+    long long* wsum = reinterpret_cast<long long*>(sm + 32);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, bid = blockIdx.x;
+    const int per = (d.R + kWarps * 32 - 1) / (kWarps * 32);
+    const int r0 = min(d.R, tid * per), r1 = min(d.R, r0 + per);
+    long long mine = 0;
+    int c16[kRowsReg], c8[kRowsReg];
 #pragma unroll
-            for (int m = 16; m >= 1; m >>= 1) L += __shfl_xor_sync(kFull, L, m);
-            tot += L * d.hkv;
-        }
-        tot = max(tot, 1ll);
-        auto F = [&](long long w) { return (int)((2 * extra * w + tot) / (2 * tot)); };
-        long long run = 0;
-        for (int b0 = 0; b0 < d.batch; b0 += 32) {
-            const int b = b0 + lane;
-            const long long L = b < d.batch ? (long long)__ldg(&p.ctx_len[b]) + p.step + 1 : 0;
-            long long incl = L;
+    for (int j = 0; j < kRowsReg; ++j) {
+        const int r = r0 + j;
+        c16[j] = r < r1 ? p.c.n_bf16[r] : 0;
+        c8[j] = r < r1 ? p.c.n_fp8[r] : 0;
+    }
+    for (int r = r0; r < r1; ++r) mine += (long long)__ldg(&p.ctx_len[r / d.hkv]) + p.step + 1;
+    long long incl = mine;
 #pragma unroll
-            for (int m = 1; m < 32; m <<= 1) {
-                const long long y = __shfl_up_sync(kFull, incl, m);
-                if (lane >= m) incl += y;
-            }
-            if (b < d.batch) {
-                long long wb = run + (incl - L) * d.hkv;   // lengths before row (b, 0)
-                for (int g = 0; g < d.hkv; ++g, wb += L) {
-                    const int r = b * d.hkv + g;
-                    const int lo = r + F(wb), hi = r + 1 + F(wb + L);
-                    if (bid >= lo && bid < hi) {
-                        sm[0] = r; sm[1] = bid - lo; sm[2] = hi - lo; sm[3] = lo;
-                    }
-                }
-            }
-            run += __shfl_sync(kFull, incl, 31) * d.hkv;
+    for (int m = 1; m < 32; m <<= 1) {
+        const long long y = __shfl_up_sync(kFull, incl, m);
+        if (lane >= m) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    long long wb = incl - mine, tot = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+        const long long x = wsum[w];
+        tot += x;
+        if (w < warp) wb += x;
+    }
+    tot = tot > 0 ? tot : 1;
+    const long long two_extra = 2ll * (gridDim.x - d.R), den = 2 * tot;
+    // the quotient from a float64 estimate (within one of it: it is at most P) and an
+    // exact integer correction, with no 64-bit division
+    auto F = [&](long long w) {
+        const long long num = two_extra * w + tot;
+        long long q = (long long)((double)num / (double)den);
+        while (q > 0 && q * den > num) --q;
+        while ((q + 1) * den <= num) ++q;
+        return (int)q;
+    };
+    for (int r = r0, j = 0; r < r1; ++r, ++j) {
+        const long long L = (long long)__ldg(&p.ctx_len[r / d.hkv]) + p.step + 1;
+        const int lo = r + F(wb), hi = r + 1 + F(wb + L);
+        if (bid >= lo && bid < hi) {
+            int n16 = 0, n8 = 0;
+#pragma unroll
+            for (int k = 0; k < kRowsReg; ++k)
+                if (k == j) { n16 = c16[k]; n8 = c8[k]; }
+            if (j >= kRowsReg) { n16 = p.c.n_bf16[r]; n8 = p.c.n_fp8[r]; }
+            out[0] = r; out[1] = bid - lo; out[2] = hi - lo; out[3] = lo; out[4] = n16; out[5] = n8;
         }
+        wb += L;
     }
     __syncthreads();
-    return Share{sm[0], sm[1], sm[2], sm[3]};
+    return Share{out[0], out[1], out[2], out[3], out[4], out[5]};
 }
 
 // The CTA's tiles: bf16 tiles [a16, e16) then FP8 tiles [a8, e8) of its row, dealt
 // round robin to the warps.  Each warp streams its tiles through its own ring of
 // kSlots slots (a bf16 tile takes two, an FP8 tile one) filled by TMA, then the CTA
 // combines its warps into one (max, sum, unnormalised o) partial in slot blockIdx.x.
+//
+// The new token's slot n16_old (when this CTA's bf16 tiles cover it: append_here)
+// is written only after the wait for the previous kernel, so the tile holding it is
+// loaded after that write; the warp that owns it stops its first fill there.
 template <int D, int FMT>
 __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int row, int n16, int n8, int a16,
-                                         int e16, int a8, int e8) {
+                                         int e16, int a8, int e8, int n16_old, bool append_here) {
     using SL = Smem<D>;
     constexpr int KB = D / 16;
     constexpr int SLOT = SL::kSlot;
@@ -524,14 +563,16 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
     auto tile_of = [&](int i) { const int li = warp + kWarps * i; return li < L16 ? a16 + li : a8 + (li - L16); };
     // producer state (every lane keeps it; lane 0 issues)
     int iss = 0, ipos = 0, free_slots = kSlots;
+    int hold = append_here ? n16_old / 16 : -1;   // the new token's tile waits for the append
     auto try_issue = [&]() {
         while (iss < nt) {
             const bool bf = iss < nt16;
             const int sz = bf ? 2 : 1;
             if (sz > free_slots) break;
+            const int jt = tile_of(iss);
+            if (bf && jt == hold) break;
             if (lane == 0) {
                 const uint32_t dst = ring + ipos * SLOT, bar = bars + 8 * ipos;
-                const int jt = tile_of(iss);
                 if (bf) {
                     const int y = row * d.cap_o + 16 * jt;
                     mbar_expect_tx(bar, 2 * SLOT);
@@ -589,6 +630,31 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
     if (!(vmax > 0.f)) vmax = 64.f;
     const float vnorm = 64.f / vmax;
 
+    // everything above read only this layer's cache and ctx_len; q, k_new, v_new and
+    // the workspace may come from the previous kernel
+    if (p.early_start) pdl_wait();
+    if (append_here) {
+        // the new token into slot n16_old, then the proxy fence and the barrier that
+        // order it before the tensor load of its tile
+        const int b = row / d.hkv, gk = row - b * d.hkv;
+        const uint16_t* kn = p.k_new + ((size_t)b * d.hkv + gk) * D;
+        const uint16_t* vn = p.v_new + ((size_t)b * d.hkv + gk) * D;
+        const size_t sl = (size_t)row * d.cap_o + n16_old;
+        for (int c = tid; c < D / 8; c += blockDim.x) {
+            *reinterpret_cast<uint4*>(p.c.k16 + sl * D + 8 * c) = *reinterpret_cast<const uint4*>(kn + 8 * c);
+            *reinterpret_cast<uint4*>(p.c.v16 + sl * D + 8 * c) = *reinterpret_cast<const uint4*>(vn + 8 * c);
+        }
+        if (tid == 0) {
+            p.c.pos16[sl] = p.ctx_len[b] + p.step;
+            p.c.mu16[sl] = 0.0;
+            p.c.m2_16[sl] = 0.0;
+        }
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncthreads();
+        hold = -1;
+        try_issue();
+    }
+
     int pos = 0;          // ring slot of the next tile to consume
     uint32_t ph = 0;      // parity of every slot's next phase
     bool aborted = false;
@@ -639,18 +705,20 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
         const int s1 = min(n8, e8 * 16);
         for (int i = nt16; i < nt; ++i) {
             const int t0 = 16 * tile_of(i);
+            // scales of this lane's tokens; zero past the segment end, where P is zero and
+            // a stale scale (NaN or Inf bits included) must not reach the product p * sv
             float skv[4], svv[4];
             const int tok[4] = {t0 + 2 * t, t0 + 2 * t + 1, t0 + 8 + 2 * t, t0 + 9 + 2 * t};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int k = tok[e] - tq0;
-                if (k < kScaleTokens) {               // tokens past the segment end get stale values
-                    skv[e] = sm_sk[min(k, kScaleTokens - 1)];
-                    svv[e] = sm_sv[min(k, kScaleTokens - 1)];
-                } else {
-                    skv[e] = __ldg(skb + min(tok[e], d.cap_q - 1));
-                    svv[e] = __ldg(svb + min(tok[e], d.cap_q - 1));
+                float a = 0.f, c = 0.f;
+                if (tok[e] < s1) {
+                    if (k < kScaleTokens) { a = sm_sk[k]; c = sm_sv[k]; }
+                    else { a = __ldg(skb + tok[e]); c = __ldg(svb + tok[e]); }
                 }
+                skv[e] = a;
+                svv[e] = c;
             }
             if (!wait_tile(i)) { aborted = true; break; }
             attend_tile<D, true, FMT>(ring + pos * SLOT, off, t0, s1, hv, lo, c2, skv, svv, vnorm, logit_head, qa,
@@ -730,44 +798,56 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
 // maxima, L = sum of l_s exp((m_s - M)/sqrt(D)), o = sum of o_s exp(..) / L over
 // the row's partials (slots base .. base + n - 1), for every head of the group,
 // one warp per head (lane l owns dims 4l .. 4l+3 for D = 128, 2l, 2l+1 for D = 64).
-// Each lane weighs the partials l, l + 32, ..., and the weights reach the other
-// lanes by shuffles.  Publishes (M, L) for the score update.
+// The partials are taken kBatch at a time with every load of a batch in flight at
+// once (lane q < kBatch also loads (m, l) of partial q); a batch whose maximum
+// exceeds the running M rescales what came before.  Partials with l = 0 carry no
+// weight and do not enter M.  Publishes (M, L) for the score update.
 template <int D>
 __device__ __forceinline__ void row_merge(const AttnParams& p, int row, int base, int n) {
     constexpr int VEC = D / 32;
+    constexpr int kBatch = 16;
     const LayerDims& d = p.d;
     const int lane = threadIdx.x & 31, h = threadIdx.x >> 5;
     if (h >= d.G) return;
     const int b = row / d.hkv, gk = row - b * d.hkv;
     const float2* pml = p.part_ml + (size_t)base * 4 + h;
     const float* po = p.part_o + ((size_t)base * 4 + h) * D + VEC * lane;
-    float M = kNegInf;
-    for (int j = lane; j < n; j += 32) M = fmaxf(M, __ldcg(pml + (size_t)j * 4).x);
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, m));
-    float L = 0.f, acc[VEC];
+    float M = kNegInf, L = 0.f, acc[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-    for (int j0 = 0; j0 < n; j0 += 32) {
-        float wl = 0.f;
-        if (j0 + lane < n) {
-            const float2 ml = __ldcg(pml + (size_t)(j0 + lane) * 4);
-            wl = (ml.y > 0.f && M != kNegInf) ? exp_scaled(ml.x, M, p.inv_sqrt_d) : 0.f;
-            L = fmaf(ml.y, wl, L);
-        }
-        const int cnt = min(32, n - j0);
-#pragma unroll 8
-        for (int q = 0; q < cnt; ++q) {
-            const float w = __shfl_sync(kFull, wl, q);
+    for (int j0 = 0; j0 < n; j0 += kBatch) {
+        const int cnt = min(kBatch, n - j0);
+        const float2 ml = lane < cnt ? __ldcg(pml + (size_t)(j0 + lane) * 4) : make_float2(kNegInf, 0.f);
+        float v[kBatch][VEC];
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
             const float* src = po + (size_t)(j0 + q) * 4 * D;
             if constexpr (VEC == 4) {
-                const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
-                acc[0] = fmaf(v.x, w, acc[0]); acc[1] = fmaf(v.y, w, acc[1]);
-                acc[2] = fmaf(v.z, w, acc[2]); acc[3] = fmaf(v.w, w, acc[3]);
+                const float4 x = q < cnt ? __ldcg(reinterpret_cast<const float4*>(src)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[q][0] = x.x; v[q][1] = x.y; v[q][2] = x.z; v[q][3] = x.w;
             } else {
-                const float2 v = __ldcg(reinterpret_cast<const float2*>(src));
-                acc[0] = fmaf(v.x, w, acc[0]); acc[1] = fmaf(v.y, w, acc[1]);
+                const float2 x = q < cnt ? __ldcg(reinterpret_cast<const float2*>(src)) : make_float2(0.f, 0.f);
+                v[q][0] = x.x; v[q][1] = x.y;
             }
+        }
+        float mb = ml.y > 0.f ? ml.x : kNegInf;
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) mb = fmaxf(mb, __shfl_xor_sync(kFull, mb, m));
+        if (mb == kNegInf) continue;                            // warp-uniform: no weight in this batch
+        if (mb > M) {
+            const float sc = M == kNegInf ? 0.f : exp_scaled(M, mb, p.inv_sqrt_d);
+            L *= sc;
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[e] *= sc;
+            M = mb;
+        }
+        const float wl = ml.y > 0.f ? exp_scaled(ml.x, M, p.inv_sqrt_d) : 0.f;
+        L = fmaf(ml.y, wl, L);
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+            const float w = __shfl_sync(kFull, wl, q);
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[e] = fmaf(v[q][e], w, acc[e]);
         }
     }
 #pragma unroll
@@ -789,13 +869,18 @@ __global__ void __launch_bounds__(32 * kWarps, ARKV_MIN_CTAS) decode_attn_kernel
     __shared__ unsigned sm_ticket;
     extern __shared__ char smem_raw[];
     char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    const Share sh = grid_share(p, reinterpret_cast<int*>(smem + SL::kShare));
-    const int row = sh.row, b = row / d.hkv, gk = row - b * d.hkv;
+    pdl_launch_dependents();
+    if (tid == 0) {
+        prefetch_map(&p.tm_k16); prefetch_map(&p.tm_v16); prefetch_map(&p.tm_k8); prefetch_map(&p.tm_v8);
+    }
+    if (!p.early_start) pdl_wait();
+    const Share sh = grid_share(p, smem + SL::kShare);
+    const int row = sh.row;
 
     // the row's counts, read once by every CTA of the row; the last one to finish
     // advances n_bf16, so no CTA of the row can see the advanced count
-    const int n16_old = min(max(p.c.n_bf16[row], 0), d.cap_o);   // counts are clamped to the
-    const int n8 = min(max(p.c.n_fp8[row], 0), d.cap_q);          // capacities before any use
+    const int n16_old = min(max(sh.n16, 0), d.cap_o);   // counts are clamped to the
+    const int n8 = min(max(sh.n8, 0), d.cap_q);          // capacities before any use
     const bool append = n16_old < d.cap_o;
     const int n16 = n16_old + (append ? 1 : 0);                    // the new token included
     // this CTA's share of the row: the same fraction of each segment's 16-token tiles,
@@ -811,27 +896,12 @@ __global__ void __launch_bounds__(32 * kWarps, ARKV_MIN_CTAS) decode_attn_kernel
             for (int st = 0; st < kSlots; ++st) mbar_init(bars + 8 * st, 1);
             asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         }
-        // append: the CTA whose tiles cover the new slot stores the token before any
-        // tensor load reads that slot (the proxy fence orders the two)
-        if (append && n16_old >= 16 * a16 && n16_old < 16 * e16) {
-            const uint16_t* kn = p.k_new + ((size_t)b * d.hkv + gk) * D;
-            const uint16_t* vn = p.v_new + ((size_t)b * d.hkv + gk) * D;
-            const size_t sl = (size_t)row * d.cap_o + n16_old;
-            for (int c = tid; c < D / 8; c += blockDim.x) {
-                *reinterpret_cast<uint4*>(p.c.k16 + sl * D + 8 * c) = *reinterpret_cast<const uint4*>(kn + 8 * c);
-                *reinterpret_cast<uint4*>(p.c.v16 + sl * D + 8 * c) = *reinterpret_cast<const uint4*>(vn + 8 * c);
-            }
-            if (tid == 0) {
-                p.c.pos16[sl] = p.ctx_len[b] + p.step;
-                p.c.mu16[sl] = 0.0;
-                p.c.m2_16[sl] = 0.0;
-            }
-            asm volatile("fence.proxy.async.global;" ::: "memory");
-        }
         if (tid == 0) *reinterpret_cast<int*>(smem + SL::kAbort) = 0;
         __syncthreads();
-        cta_body<D, FMT>(p, smem, row, n16, n8, a16, e16, a8, e8);
+        const bool append_here = append && n16_old >= 16 * a16 && n16_old < 16 * e16;
+        cta_body<D, FMT>(p, smem, row, n16, n8, a16, e16, a8, e8, n16_old, append_here);
     } else {
+        if (p.early_start) pdl_wait();
         for (int idx = tid; idx < 4 * D; idx += blockDim.x) {   // nothing to attend: an empty partial
             p.part_o[(size_t)blockIdx.x * 4 * D + idx] = 0.f;
             if (idx < 4) p.part_ml[(size_t)blockIdx.x * 4 + idx] = make_float2(kNegInf, 0.f);
@@ -980,8 +1050,19 @@ cudaError_t launch_decode_attn(AttnParams& p, cudaStream_t s) {
         P = P < units / 16 ? P : units / 16;
         if (P > kMaxGrid) P = kMaxGrid;
         if (P < d.R) P = d.R;
-        kernel<<<dim3((unsigned)P), 32 * kWarps, bytes, s>>>(p);
-        return cudaSuccess;
+        // a programmatic dependent of the previous kernel on the stream (the kernel
+        // waits for it with griddepcontrol.wait before it reads what that kernel may write)
+        cudaLaunchConfig_t lc{};
+        lc.gridDim = dim3((unsigned)P);
+        lc.blockDim = dim3(32 * kWarps);
+        lc.dynamicSmemBytes = (size_t)bytes;
+        lc.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        lc.attrs = attr;
+        lc.numAttrs = 1;
+        return cudaLaunchKernelEx(&lc, kernel, p);
     };
     if (D == 128)
         e = d.fmt == ARKV_FMT_E5M2 ? go(decode_attn_kernel<128, ARKV_FMT_E5M2>, 0, Smem<128>::kBytes)

@@ -43,7 +43,7 @@ def test_oq_ratio_matches_oracle(lib):
 
 def cfg(**kw):
     base = dict(batch=1, hq=8, hkv=2, head_dim=64, window=64, n_obs=64, gamma=1.0, budget_frac=0.25,
-                cap_bf16=1000, cap_fp8=1000, quant_format=abi.ARKV_FMT_E4M3)
+                cap_bf16=1000, cap_fp8=1000, quant_format=abi.ARKV_FMT_E4M3, early_start=0)
     base.update(kw)
     return abi.arkv_cfg(*[base[n] for n, _ in abi.arkv_cfg._fields_])
 
@@ -68,7 +68,8 @@ def test_workspace_sizes(lib):
 
 @pytest.mark.parametrize("bad", [dict(head_dim=96), dict(hq=7), dict(hq=16, hkv=2), dict(window=0),
                                  dict(budget_frac=0.0), dict(budget_frac=1.5), dict(gamma=-1.0),
-                                 dict(cap_fp8=0), dict(quant_format=2), dict(quant_format=-1)])
+                                 dict(cap_fp8=0), dict(quant_format=2), dict(quant_format=-1),
+                                 dict(early_start=2), dict(early_start=-1)])
 def test_bad_config_rejected_before_launch(lib, bad):
     c = cfg(**bad)
     dummy = ctypes.c_void_p(256)

@@ -135,6 +135,7 @@ def run_scenario(wl, steps, dev, rows=None, r=None, kernel_parity=False, seed=0,
         dl.decode(t, to_dev(d["q"], dev), to_dev(d["k_new"], dev), to_dev(d["v_new"], dev), ctx_t, o)
         dl.score(t, ctx_t)
         og = o.cpu().numpy()
+        assert np.isfinite(og).all(), (t, np.argwhere(~np.isfinite(og).all(-1)).tolist()[:8])  # every row, not only the compared ones
         for rid in rows:
             b, g = divmod(rid, wl.hkv)
             sl = slice(g * wl.group, (g + 1) * wl.group)
