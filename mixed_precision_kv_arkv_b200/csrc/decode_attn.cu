@@ -4,10 +4,11 @@
 //
 // One wave of CTAs (as many as the GPU holds at once) shares the rows in
 // proportion to their lengths; each CTA takes the same fraction of its row's bf16
-// tiles and of its FP8 tiles (16 tokens each), bf16 tiles first.  Its 4 warps take the tiles round robin, each through its
-// own ring of 4 shared-memory slots (a bf16 tile takes two, K then V; an FP8 tile
-// one) filled by TMA tensor loads (16 rows per box, 128-byte swizzle; 64-byte for
-// FP8 rows of 64 bytes) completing on per-slot mbarriers (waits are bounded).
+// tiles and of its FP8 tiles (16 tokens each), bf16 tiles first.  Its 4 warps take
+// the tiles round robin, each through its own ring of 4 shared-memory slots (a bf16
+// tile takes two, K then V; an FP8 tile one) filled by TMA tensor loads (16 rows per
+// box, 128-byte swizzle; 64-byte for FP8 rows of 64 bytes) completing on per-slot
+// mbarriers (waits are bounded).
 //
 // Tile math on the warp-level tensor cores (m16n8k16).  QK^T with the queries as
 // the M rows: rows 0..3 and 4..7 both hold the group's heads (zero past G), rows
@@ -27,16 +28,16 @@
 //   4t..4t+3 supplied, and the rows are supplied in the token order 0,1,8,9,
 //   2,3,10,11, ... so that they are tokens 2t, 2t+1, 8+2t, 9+2t -- the k positions
 //   of the bf16 path.  The per-token K scale multiplies the finished logit; the V
-//   scale is folded into P, and every tile's P is multiplied by 64 / (the largest V
-//   scale of the warp's FP8 tiles), which keeps p * sv inside f16 and comes back
-//   out of the partial.
+//   scale is folded into P, and P is multiplied by 64 / (the largest V scale of
+//   the warp's FP8 tiles so far; the accumulator is rescaled when it grows), which
+//   keeps p * sv inside f16 and comes back out of the partial.
 // Softmax in float32 with a reference maximum that moves only when a logit
 // exceeds it by 2^8 (so most tiles need no reduction, which is two shuffles over
 // the 4 lanes of a row when it happens).  Raw logits go to the workspace for the
 // score update.  The CTA combines its warps into one (max, sum, unnormalised o)
 // partial; the last CTA of a row to finish (a ticket in the workspace) merges the
-// row's partials into o and each head's final (max, sum), and advances the row's
-// bf16 count past the appended token.
+// row's partials and the new token into o and each head's final (max, sum), stores
+// the new token in the cache and advances the row's bf16 count past it.
 #include <math.h>
 #include <mutex>
 
@@ -55,14 +56,13 @@ constexpr unsigned kFull = 0xffffffffu;
 #define ARKV_MIN_CTAS 3
 #endif
 #ifndef ARKV_QK_CHAINS
-#define ARKV_QK_CHAINS 2
+#define ARKV_QK_CHAINS 1
 #endif
 constexpr int kQkChains = ARKV_QK_CHAINS;   // independent QK^T accumulator chains per n-tile
 constexpr int kWarps = 4;
 constexpr int kSlots = 4;                  // ring slots per warp: a bf16 tile takes 2, an FP8 tile 1
 constexpr int kSpinLimit = 1 << 20;        // bounded mbarrier waits (~1 s worst case)
 constexpr int kMaxGrid = 2048;             // CTAs of one call at most (partial slots in the workspace)
-constexpr int kScaleTokens = 512;          // FP8 scales a CTA keeps in shared memory (the rest from L2)
 
 // ------------------------------------------------------------------ shared-memory layout
 template <int D>
@@ -76,9 +76,10 @@ struct Smem {
     static constexpr int kMax = kRed + 16 * 4;                          // float [4]
     static constexpr int kAbort = kMax + 16;                            // int: a wait gave up
     static constexpr int kShare = kAbort + 16;                          // int [8] + int64 [4]: grid share
-    static constexpr int kScales = kShare + 64;                         // float [2][kScaleTokens]: sk, sv
-    static constexpr int kVmax = kScales + 2 * kScaleTokens * 4;        // float [4]
-    static constexpr int kBytes = kVmax + 16 + 1024;                    // + alignment slack
+    static constexpr int kTileq = kShare + 64;                          // int [4][kSlots]: tile of each slot
+    static constexpr int kSc = kTileq + kWarps * kSlots * 4;            // float [4][kSlots][32]: FP8 scales
+    static constexpr int kQ = kSc + kWarps * kSlots * 32 * 4;           // bf16 [4][D]: the group's queries
+    static constexpr int kBytes = kQ + 4 * D * 2 + 1024;                // + alignment slack
     static constexpr int kO = 0;                                        // float [4][4][D], in the idle ring
     static_assert(4 * 4 * D * 4 <= kRing, "the epilogue buffer must fit in the ring");
 };
@@ -158,6 +159,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
 // before this one has finished with its writes visible.
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// 4-byte asynchronous copy global -> shared (one cp.async group per commit).
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ void prefetch_map(const CUtensorMap* m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -433,26 +442,23 @@ __device__ __forceinline__ void attend_tile(uint32_t st, const LaneOffsets<D, FP
 }
 
 // A fragments (a0, a2 of every k block) of query row g: head g & 3 (rows 0..3 and
-// 4..7 repeat the group; zero for heads >= G): bf16 in natural dimension order;
-// f16 for FP8 tiles, in the order of the 4-byte K words (dims 16 kk + 4t .. + 3).
+// 4..7 repeat the group; the rows of heads >= G are zero in qs): bf16 in natural
+// dimension order; f16 for FP8 tiles, in the order of the 4-byte K words (dims
+// 16 kk + 4t .. + 3).  qs: the group's queries in shared memory, [4][D] bf16.
 template <int D>
-__device__ __forceinline__ void load_q(const AttnParams& p, int row, bool fp8, uint32_t (&qa)[D / 16][2]) {
+__device__ __forceinline__ void load_q(const uint16_t* qs, bool fp8, uint32_t (&qa)[D / 16][2]) {
     const int lane = threadIdx.x & 31, h = (lane >> 2) & 3, t = lane & 3;
-    const int b = row / p.d.hkv, gk = row - b * p.d.hkv, G = p.d.G;
-    const bool hv = h < G;
-    const uint16_t* qrow = p.q + ((size_t)b * p.d.hq + gk * G + (hv ? h : 0)) * D;
+    const uint16_t* qrow = qs + h * D;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t x = 0u, y = 0u;
-        if (hv) {
-            if (fp8) {
-                const uint2 u = *reinterpret_cast<const uint2*>(qrow + 16 * kk + 4 * t);
-                x = pack_f16(bf16_lo(u.x), bf16_hi(u.x));
-                y = pack_f16(bf16_lo(u.y), bf16_hi(u.y));
-            } else {
-                x = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * t);
-                y = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * t + 8);
-            }
+        uint32_t x, y;
+        if (fp8) {
+            const uint2 u = *reinterpret_cast<const uint2*>(qrow + 16 * kk + 4 * t);
+            x = pack_f16(bf16_lo(u.x), bf16_hi(u.x));
+            y = pack_f16(bf16_lo(u.y), bf16_hi(u.y));
+        } else {
+            x = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * t);
+            y = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * t + 8);
         }
         qa[kk][0] = x;
         qa[kk][1] = y;
@@ -535,17 +541,25 @@ __device__ __forceinline__ Share grid_share(const AttnParams& p, char* sm) {
     return Share{out[0], out[1], out[2], out[3], out[4], out[5]};
 }
 
-// The CTA's tiles: bf16 tiles [a16, e16) then FP8 tiles [a8, e8) of its row, dealt
-// round robin to the warps.  Each warp streams its tiles through its own ring of
-// kSlots slots (a bf16 tile takes two, an FP8 tile one) filled by TMA, then the CTA
+// The CTA's tiles: bf16 tiles [a16, e16) then FP8 tiles [a8, e8) of its row (16
+// tokens each), dealt round robin to the warps.  Each warp streams its tiles through
+// its own ring of kSlots slots (a bf16 tile takes two, an FP8 tile one) filled by
+// TMA; an FP8 tile's 16 K and 16 V scales come with it, one 4-byte cp.async per lane
+// into the slot's scale area (one cp.async group per issued tile).  The CTA then
 // combines its warps into one (max, sum, unnormalised o) partial in slot blockIdx.x.
 //
-// The new token's slot n16_old (when this CTA's bf16 tiles cover it: append_here)
-// is written only after the wait for the previous kernel, so the tile holding it is
-// loaded after that write; the warp that owns it stops its first fill there.
+// With early_start the warps fill their rings before the wait for the previous
+// kernel, so that this call's cache starts streaming while that kernel finishes.
+// The tiles cover the row's tokens before this call's append; the new token is
+// attended by the row's merge.
+//
+// The V scale is folded into P in f16, so P is also multiplied by vnorm = 64 / (the
+// largest V scale among the warp's FP8 tiles so far): p sv vnorm <= 2^8 * 64 stays
+// inside f16 and well above its subnormals.  vnorm starts at 1 and the accumulator
+// is rescaled when an FP8 tile raises the maximum; it comes back out of the partial.
 template <int D, int FMT>
 __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int row, int n16, int n8, int a16,
-                                         int e16, int a8, int e8, int n16_old, bool append_here) {
+                                         int e16, int a8, int e8) {
     using SL = Smem<D>;
     constexpr int KB = D / 16;
     constexpr int SLOT = SL::kSlot;
@@ -555,25 +569,31 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
     const uint32_t ring = sbase + warp * kSlots * SLOT;
     const uint32_t bars = sbase + SL::kBars + warp * kSlots * 8;
     int* sm_abort = reinterpret_cast<int*>(smem + SL::kAbort);
+    int* sm_tq = reinterpret_cast<int*>(smem + SL::kTileq) + warp * kSlots;      // (tile << 1) | fp8, by slot
+    float* sm_sc = reinterpret_cast<float*>(smem + SL::kSc) + warp * kSlots * 32;  // scales, by slot
+    uint16_t* sm_q = reinterpret_cast<uint16_t*>(smem + SL::kQ);                  // [4][D] bf16
+    const uint32_t sc_base = smem_u32(sm_sc);
+    const int b = row / d.hkv, gk = row - b * d.hkv;
 
     // this warp's tiles: list positions warp, warp + 4, ... of [bf16 tiles, FP8 tiles]
     const int L16 = e16 - a16, L = L16 + (e8 - a8);
     const int nt16 = L16 > warp ? (L16 - warp + kWarps - 1) / kWarps : 0;
     const int nt = L > warp ? (L - warp + kWarps - 1) / kWarps : 0;
-    auto tile_of = [&](int i) { const int li = warp + kWarps * i; return li < L16 ? a16 + li : a8 + (li - L16); };
-    // producer state (every lane keeps it; lane 0 issues)
+    auto enc_of = [&](int i) {   // the warp's i-th tile: (tile << 1) | fp8
+        const int li = warp + kWarps * i;
+        return li < L16 ? (a16 + li) << 1 : ((a8 + li - L16) << 1) | 1;
+    };
+    // producer state (every lane keeps it; lane 0 issues the tensor loads)
     int iss = 0, ipos = 0, free_slots = kSlots;
-    int hold = append_here ? n16_old / 16 : -1;   // the new token's tile waits for the append
     auto try_issue = [&]() {
         while (iss < nt) {
-            const bool bf = iss < nt16;
-            const int sz = bf ? 2 : 1;
+            const int enc = enc_of(iss);
+            const bool f8 = enc & 1;
+            const int jt = enc >> 1, sz = f8 ? 1 : 2;
             if (sz > free_slots) break;
-            const int jt = tile_of(iss);
-            if (bf && jt == hold) break;
+            const uint32_t dst = ring + ipos * SLOT, bar = bars + 8 * ipos;
             if (lane == 0) {
-                const uint32_t dst = ring + ipos * SLOT, bar = bars + 8 * ipos;
-                if (bf) {
+                if (!f8) {
                     const int y = row * d.cap_o + 16 * jt;
                     mbar_expect_tx(bar, 2 * SLOT);
 #pragma unroll
@@ -588,6 +608,13 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
                     tma_load_2d(dst + 16 * D, &p.tm_v8, 0, y, bar);
                 }
             }
+            if (f8) {   // lanes 0..15: K scales of the tile's tokens, 16..31: V scales
+                const int tok = min(16 * jt + (lane & 15), d.cap_q - 1);
+                cp_async4(sc_base + (ipos * 32 + lane) * 4,
+                          (lane < 16 ? p.c.sk : p.c.sv) + (size_t)row * d.cap_q + tok);
+            }
+            cp_async_commit();
+            sm_tq[ipos] = enc;
             ipos = (ipos + sz) & (kSlots - 1);
             free_slots -= sz;
             ++iss;
@@ -603,62 +630,22 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
 #pragma unroll
     for (int mt = 0; mt < KB; ++mt) oacc[mt][0] = oacc[mt][1] = oacc[mt][2] = oacc[mt][3] = 0.f;
 
-    // the CTA's FP8 scales: the first kScaleTokens into shared memory, one coalesced
-    // pass by the whole CTA that also finds the largest V scale (64 if there is none);
-    // every tile's P is multiplied by vnorm = 64 / vmax (p < 2^8: p sv vnorm < 2^14,
-    // inside f16)
-    const float* skb = p.c.sk + (size_t)row * d.cap_q;
-    const float* svb = p.c.sv + (size_t)row * d.cap_q;
-    float* sm_sk = reinterpret_cast<float*>(smem + SL::kScales);
-    float* sm_sv = sm_sk + kScaleTokens;
-    float* sm_vmax = reinterpret_cast<float*>(smem + SL::kVmax);
-    const int tq0 = 16 * a8, tq1 = min(16 * e8, n8);
-    float vm = 0.f;
-    for (int k = tq0 + tid; k < tq1; k += blockDim.x) {
-        const float v = __ldg(svb + k);
-        vm = fmaxf(vm, v);
-        if (k - tq0 < kScaleTokens) {
-            sm_sk[k - tq0] = __ldg(skb + k);
-            sm_sv[k - tq0] = v;
-        }
-    }
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) vm = fmaxf(vm, __shfl_xor_sync(kFull, vm, m));
-    if (lane == 0) sm_vmax[warp] = vm;
-    __syncthreads();
-    float vmax = fmaxf(fmaxf(sm_vmax[0], sm_vmax[1]), fmaxf(sm_vmax[2], sm_vmax[3]));
-    if (!(vmax > 0.f)) vmax = 64.f;
-    const float vnorm = 64.f / vmax;
-
     // everything above read only this layer's cache and ctx_len; q, k_new, v_new and
     // the workspace may come from the previous kernel
     if (p.early_start) pdl_wait();
-    if (append_here) {
-        // the new token into slot n16_old, then the proxy fence and the barrier that
-        // order it before the tensor load of its tile
-        const int b = row / d.hkv, gk = row - b * d.hkv;
-        const uint16_t* kn = p.k_new + ((size_t)b * d.hkv + gk) * D;
-        const uint16_t* vn = p.v_new + ((size_t)b * d.hkv + gk) * D;
-        const size_t sl = (size_t)row * d.cap_o + n16_old;
-        for (int c = tid; c < D / 8; c += blockDim.x) {
-            *reinterpret_cast<uint4*>(p.c.k16 + sl * D + 8 * c) = *reinterpret_cast<const uint4*>(kn + 8 * c);
-            *reinterpret_cast<uint4*>(p.c.v16 + sl * D + 8 * c) = *reinterpret_cast<const uint4*>(vn + 8 * c);
-        }
-        if (tid == 0) {
-            p.c.pos16[sl] = p.ctx_len[b] + p.step;
-            p.c.mu16[sl] = 0.0;
-            p.c.m2_16[sl] = 0.0;
-        }
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-        __syncthreads();
-        hold = -1;
-        try_issue();
+    for (int i = tid; i < 4 * D / 8; i += blockDim.x) {   // the group's queries, zero past G
+        const int h = i / (D / 8), c = i - h * (D / 8);
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (h < d.G) v = *reinterpret_cast<const uint4*>(p.q + ((size_t)b * d.hq + gk * d.G + h) * D + 8 * c);
+        *reinterpret_cast<uint4*>(sm_q + h * D + 8 * c) = v;
     }
+    __syncthreads();
 
     int pos = 0;          // ring slot of the next tile to consume
     uint32_t ph = 0;      // parity of every slot's next phase
+    int cons = 0;         // tiles consumed
     bool aborted = false;
-    auto wait_tile = [&](int i) -> bool {
+    auto wait_tile = [&]() -> bool {
         if (mbar_wait(bars + 8 * pos, (ph >> pos) & 1u)) return true;
         // a copy did not land in time: flag it, give every copy this warp has in flight
         // (this one included) a last bounded chance to land, and leave the ring alone
@@ -667,10 +654,10 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
             atomicExch(sm_abort, 1);
         }
         uint32_t q = ph;
-        for (int j = i, sp = pos; j < iss; ++j) {
+        for (int j = cons, sp = pos; j < iss; ++j) {
             mbar_wait(bars + 8 * sp, (q >> sp) & 1u);
             q ^= 1u << sp;
-            sp = (sp + (j < nt16 ? 2 : 1)) & (kSlots - 1);
+            sp = (sp + ((sm_tq[sp] & 1) ? 1 : 2)) & (kSlots - 1);
         }
         return false;
     };
@@ -678,54 +665,72 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
         ph ^= 1u << pos;
         pos = (pos + sz) & (kSlots - 1);
         free_slots += sz;
+        ++cons;
         __syncwarp();
         try_issue();
     };
 
-    // ---- bf16 tiles
     uint32_t qa[KB][2];
+    float vnorm = 1.f, vcur = 0.f;   // vcur: the largest V scale seen, 0 before any FP8 tile
+    // ---- bf16 tiles
     if (nt16 > 0) {
-        load_q<D>(p, row, false, qa);
+        load_q<D>(sm_q, false, qa);
         const LaneOffsets<D, false> off;
         float* logit_head = p.logit16 + ((size_t)row * 4 + (hv ? hd : 0)) * p.lstride_o;
         const float one[4] = {1.f, 1.f, 1.f, 1.f};
-        const int s1 = min(n16, e16 * 16);
         for (int i = 0; i < nt16; ++i) {
-            if (!wait_tile(i)) { aborted = true; break; }
-            attend_tile<D, false, FMT>(ring + pos * SLOT, off, 16 * tile_of(i), s1, hv, lo, c2, one, one, vnorm,
-                                       logit_head, qa, rs, oacc);
+            const int t0 = 16 * (sm_tq[pos] >> 1);
+            if (!wait_tile()) { aborted = true; break; }
+            attend_tile<D, false, FMT>(ring + pos * SLOT, off, t0, n16, hv, lo, c2, one, one, 1.f, logit_head, qa,
+                                       rs, oacc);
             release(2);
         }
     }
-    // ---- FP8 tiles, their scales loaded one tile ahead
+    // ---- FP8 tiles
     if (!aborted && nt > nt16) {
-        load_q<D>(p, row, true, qa);
+        load_q<D>(sm_q, true, qa);
         const LaneOffsets<D, true> off;
         float* logit_head = p.logit8 + ((size_t)row * 4 + (hv ? hd : 0)) * p.lstride_q;
-        const int s1 = min(n8, e8 * 16);
         for (int i = nt16; i < nt; ++i) {
-            const int t0 = 16 * tile_of(i);
+            const int t0 = 16 * (sm_tq[pos] >> 1);
+            if (!wait_tile()) { aborted = true; break; }
+            // this tile's scale group (the groups of later tiles may still be in flight)
+            switch (iss - cons - 1) {
+                case 0: cp_async_wait<0>(); break;
+                case 1: cp_async_wait<1>(); break;
+                case 2: cp_async_wait<2>(); break;
+                default: cp_async_wait<3>(); break;
+            }
+            __syncwarp();
             // scales of this lane's tokens; zero past the segment end, where P is zero and
             // a stale scale (NaN or Inf bits included) must not reach the product p * sv
+            const float* sc = sm_sc + pos * 32;
             float skv[4], svv[4];
-            const int tok[4] = {t0 + 2 * t, t0 + 2 * t + 1, t0 + 8 + 2 * t, t0 + 9 + 2 * t};
+            const int tk[4] = {2 * t, 2 * t + 1, 8 + 2 * t, 9 + 2 * t};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int k = tok[e] - tq0;
-                float a = 0.f, c = 0.f;
-                if (tok[e] < s1) {
-                    if (k < kScaleTokens) { a = sm_sk[k]; c = sm_sv[k]; }
-                    else { a = __ldg(skb + tok[e]); c = __ldg(svb + tok[e]); }
-                }
-                skv[e] = a;
-                svv[e] = c;
+                const bool ok = t0 + tk[e] < n8;
+                skv[e] = ok ? sc[tk[e]] : 0.f;
+                svv[e] = ok ? sc[16 + tk[e]] : 0.f;
             }
-            if (!wait_tile(i)) { aborted = true; break; }
-            attend_tile<D, true, FMT>(ring + pos * SLOT, off, t0, s1, hv, lo, c2, skv, svv, vnorm, logit_head, qa,
+            float m = fmaxf(fmaxf(svv[0], svv[1]), fmaxf(svv[2], svv[3]));
+            m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));   // the tile's largest V scale (every lane)
+            if (m > vcur) {
+                const float vn = 64.f / m, f = vn / vnorm;
+#pragma unroll
+                for (int mt = 0; mt < KB; ++mt) {
+                    oacc[mt][0] *= f; oacc[mt][1] *= f; oacc[mt][2] *= f; oacc[mt][3] *= f;
+                }
+                vnorm = vn;
+                vcur = m;
+            }
+            attend_tile<D, true, FMT>(ring + pos * SLOT, off, t0, n8, hv, lo, c2, skv, svv, vnorm, logit_head, qa,
                                       rs, oacc);
             release(1);
         }
     }
+    cp_async_wait<0>();
 
     __syncthreads();   // every warp has drained its ring: the epilogue may reuse it
     const size_t pb = blockIdx.x;
@@ -751,7 +756,7 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
     float l = rs.l;
     l += __shfl_xor_sync(kFull, l, 1);
     l += __shfl_xor_sync(kFull, l, 2);
-    const float un = vmax * (1.f / 64.f);
+    const float un = vcur > 0.f ? vcur * (1.f / 64.f) : 1.f;   // 1 / vnorm
 #pragma unroll
     for (int mt = 0; mt < KB; ++mt)
 #pragma unroll
@@ -801,9 +806,15 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
 // The partials are taken kBatch at a time with every load of a batch in flight at
 // once (lane q < kBatch also loads (m, l) of partial q); a batch whose maximum
 // exceeds the running M rescales what came before.  Partials with l = 0 carry no
-// weight and do not enter M.  Publishes (M, L) for the score update.
+// weight and do not enter M.
+// The new token (slot s_new >= 0; -1: the bf16 segment is full and the token is
+// dropped) enters here as one more term: its logit q . k_new (float32 products of
+// the bf16 values, summed over the warp), its weight exp((q.k - M')/sqrt(D)) and
+// its value v_new; its raw logit goes to the workspace with the others, and the
+// token is stored in slot s_new for later calls (no tensor load of this call reads
+// that slot).  Publishes (M, L) for the score update.
 template <int D>
-__device__ __forceinline__ void row_merge(const AttnParams& p, int row, int base, int n) {
+__device__ __forceinline__ void row_merge(const AttnParams& p, int row, int base, int n, int s_new) {
     constexpr int VEC = D / 32;
     constexpr int kBatch = 16;
     const LayerDims& d = p.d;
@@ -852,6 +863,53 @@ __device__ __forceinline__ void row_merge(const AttnParams& p, int row, int base
     }
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) L += __shfl_xor_sync(kFull, L, m);
+    if (s_new >= 0) {
+        const uint16_t* qh = p.q + ((size_t)b * d.hq + gk * d.G + h) * D + VEC * lane;
+        const uint16_t* kn = p.k_new + ((size_t)b * d.hkv + gk) * D + VEC * lane;
+        const uint16_t* vn = p.v_new + ((size_t)b * d.hkv + gk) * D + VEC * lane;
+        float kv[VEC], vv[VEC], qv[VEC];
+        if constexpr (VEC == 4) {
+            const uint2 q2 = *reinterpret_cast<const uint2*>(qh), k2 = *reinterpret_cast<const uint2*>(kn),
+                        v2 = *reinterpret_cast<const uint2*>(vn);
+            qv[0] = bf16_lo(q2.x); qv[1] = bf16_hi(q2.x); qv[2] = bf16_lo(q2.y); qv[3] = bf16_hi(q2.y);
+            kv[0] = bf16_lo(k2.x); kv[1] = bf16_hi(k2.x); kv[2] = bf16_lo(k2.y); kv[3] = bf16_hi(k2.y);
+            vv[0] = bf16_lo(v2.x); vv[1] = bf16_hi(v2.x); vv[2] = bf16_lo(v2.y); vv[3] = bf16_hi(v2.y);
+        } else {
+            const uint32_t q1 = *reinterpret_cast<const uint32_t*>(qh), k1 = *reinterpret_cast<const uint32_t*>(kn),
+                           v1 = *reinterpret_cast<const uint32_t*>(vn);
+            qv[0] = bf16_lo(q1); qv[1] = bf16_hi(q1);
+            kv[0] = bf16_lo(k1); kv[1] = bf16_hi(k1);
+            vv[0] = bf16_lo(v1); vv[1] = bf16_hi(v1);
+        }
+        float sdot = 0.f;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) sdot = fmaf(qv[e], kv[e], sdot);
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) sdot += __shfl_xor_sync(kFull, sdot, m);
+        const float Mn = fmaxf(M, sdot);
+        const float sc = M == kNegInf ? 0.f : exp_scaled(M, Mn, p.inv_sqrt_d);
+        const float wn = exp_scaled(sdot, Mn, p.inv_sqrt_d);
+        L = fmaf(L, sc, wn);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] = fmaf(acc[e], sc, wn * vv[e]);
+        M = Mn;
+        if (lane == 0) p.logit16[((size_t)row * 4 + h) * p.lstride_o + s_new] = sdot;
+        if (h == 0) {   // the token into slot s_new for the calls that follow
+            const size_t s16 = (size_t)row * d.cap_o + s_new;
+            if constexpr (VEC == 4) {
+                *reinterpret_cast<uint2*>(p.c.k16 + s16 * D + VEC * lane) = *reinterpret_cast<const uint2*>(kn);
+                *reinterpret_cast<uint2*>(p.c.v16 + s16 * D + VEC * lane) = *reinterpret_cast<const uint2*>(vn);
+            } else {
+                *reinterpret_cast<uint32_t*>(p.c.k16 + s16 * D + VEC * lane) = *reinterpret_cast<const uint32_t*>(kn);
+                *reinterpret_cast<uint32_t*>(p.c.v16 + s16 * D + VEC * lane) = *reinterpret_cast<const uint32_t*>(vn);
+            }
+            if (lane == 0) {
+                p.c.pos16[s16] = p.ctx_len[b] + p.step;
+                p.c.mu16[s16] = 0.0;
+                p.c.m2_16[s16] = 0.0;
+            }
+        }
+    }
     float* out = p.o + ((size_t)b * d.hq + gk * d.G + h) * D + VEC * lane;
     const float inv = 1.f / L;
     if constexpr (VEC == 4)
@@ -879,10 +937,9 @@ __global__ void __launch_bounds__(32 * kWarps, ARKV_MIN_CTAS) decode_attn_kernel
 
     // the row's counts, read once by every CTA of the row; the last one to finish
     // advances n_bf16, so no CTA of the row can see the advanced count
-    const int n16_old = min(max(sh.n16, 0), d.cap_o);   // counts are clamped to the
-    const int n8 = min(max(sh.n8, 0), d.cap_q);          // capacities before any use
-    const bool append = n16_old < d.cap_o;
-    const int n16 = n16_old + (append ? 1 : 0);                    // the new token included
+    const int n16 = min(max(sh.n16, 0), d.cap_o);   // counts are clamped to the
+    const int n8 = min(max(sh.n8, 0), d.cap_q);      // capacities before any use
+    const bool append = n16 < d.cap_o;               // the new token goes to slot n16
     // this CTA's share of the row: the same fraction of each segment's 16-token tiles,
     // so that every CTA of the row has the same mix of bf16 and FP8 work
     const int T16 = (n16 + 15) / 16, T8 = (n8 + 15) / 16;
@@ -898,8 +955,7 @@ __global__ void __launch_bounds__(32 * kWarps, ARKV_MIN_CTAS) decode_attn_kernel
         }
         if (tid == 0) *reinterpret_cast<int*>(smem + SL::kAbort) = 0;
         __syncthreads();
-        const bool append_here = append && n16_old >= 16 * a16 && n16_old < 16 * e16;
-        cta_body<D, FMT>(p, smem, row, n16, n8, a16, e16, a8, e8, n16_old, append_here);
+        cta_body<D, FMT>(p, smem, row, n16, n8, a16, e16, a8, e8);
     } else {
         if (p.early_start) pdl_wait();
         for (int idx = tid; idx < 4 * D; idx += blockDim.x) {   // nothing to attend: an empty partial
@@ -916,10 +972,10 @@ __global__ void __launch_bounds__(32 * kWarps, ARKV_MIN_CTAS) decode_attn_kernel
     __syncthreads();
     if (sm_ticket != (unsigned)(sh.n - 1)) return;
     __threadfence();
-    row_merge<D>(p, row, sh.base, sh.n);
+    row_merge<D>(p, row, sh.base, sh.n, append ? n16 : -1);
     if (tid == 0) {
         p.counter[row] = 0u;                                   // ready for the next call
-        if (append) p.c.n_bf16[row] = n16_old + 1;
+        if (append) p.c.n_bf16[row] = n16 + 1;
         else atomicOr(p.c.status, ARKV_STATUS_BF16_FULL);      // the new token was dropped
     }
 }
