@@ -60,6 +60,10 @@ constexpr unsigned kFull = 0xffffffffu;
 #endif
 constexpr int kQkChains = ARKV_QK_CHAINS;   // independent QK^T accumulator chains per n-tile
 constexpr int kWarps = 4;
+#ifndef ARKV_GRID_RESERVE
+#define ARKV_GRID_RESERVE 1
+#endif
+constexpr bool kGridReserve = ARKV_GRID_RESERVE != 0;
 constexpr int kSlots = 4;                  // ring slots per warp: a bf16 tile takes 2, an FP8 tile 1
 constexpr int kSpinLimit = 1 << 20;        // bounded mbarrier waits (~1 s worst case)
 constexpr int kMaxGrid = 2048;             // CTAs of one call at most (partial slots in the workspace)
@@ -823,6 +827,20 @@ __device__ __forceinline__ void row_merge(const AttnParams& p, int row, int base
     const int b = row / d.hkv, gk = row - b * d.hkv;
     const float2* pml = p.part_ml + (size_t)base * 4 + h;
     const float* po = p.part_o + ((size_t)base * 4 + h) * D + VEC * lane;
+    // the new token's query, key and value dims of this lane, loaded with the first batch
+    const uint16_t* qh = p.q + ((size_t)b * d.hq + gk * d.G + h) * D + VEC * lane;
+    const uint16_t* kn = p.k_new + ((size_t)b * d.hkv + gk) * D + VEC * lane;
+    const uint16_t* vn = p.v_new + ((size_t)b * d.hkv + gk) * D + VEC * lane;
+    uint2 q2 = make_uint2(0u, 0u), k2 = q2, v2 = q2;
+    if (s_new >= 0) {
+        if constexpr (VEC == 4) {
+            q2 = *reinterpret_cast<const uint2*>(qh); k2 = *reinterpret_cast<const uint2*>(kn);
+            v2 = *reinterpret_cast<const uint2*>(vn);
+        } else {
+            q2.x = *reinterpret_cast<const uint32_t*>(qh); k2.x = *reinterpret_cast<const uint32_t*>(kn);
+            v2.x = *reinterpret_cast<const uint32_t*>(vn);
+        }
+    }
     float M = kNegInf, L = 0.f, acc[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
@@ -864,22 +882,14 @@ __device__ __forceinline__ void row_merge(const AttnParams& p, int row, int base
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) L += __shfl_xor_sync(kFull, L, m);
     if (s_new >= 0) {
-        const uint16_t* qh = p.q + ((size_t)b * d.hq + gk * d.G + h) * D + VEC * lane;
-        const uint16_t* kn = p.k_new + ((size_t)b * d.hkv + gk) * D + VEC * lane;
-        const uint16_t* vn = p.v_new + ((size_t)b * d.hkv + gk) * D + VEC * lane;
         float kv[VEC], vv[VEC], qv[VEC];
+        qv[0] = bf16_lo(q2.x); qv[1] = bf16_hi(q2.x);
+        kv[0] = bf16_lo(k2.x); kv[1] = bf16_hi(k2.x);
+        vv[0] = bf16_lo(v2.x); vv[1] = bf16_hi(v2.x);
         if constexpr (VEC == 4) {
-            const uint2 q2 = *reinterpret_cast<const uint2*>(qh), k2 = *reinterpret_cast<const uint2*>(kn),
-                        v2 = *reinterpret_cast<const uint2*>(vn);
-            qv[0] = bf16_lo(q2.x); qv[1] = bf16_hi(q2.x); qv[2] = bf16_lo(q2.y); qv[3] = bf16_hi(q2.y);
-            kv[0] = bf16_lo(k2.x); kv[1] = bf16_hi(k2.x); kv[2] = bf16_lo(k2.y); kv[3] = bf16_hi(k2.y);
-            vv[0] = bf16_lo(v2.x); vv[1] = bf16_hi(v2.x); vv[2] = bf16_lo(v2.y); vv[3] = bf16_hi(v2.y);
-        } else {
-            const uint32_t q1 = *reinterpret_cast<const uint32_t*>(qh), k1 = *reinterpret_cast<const uint32_t*>(kn),
-                           v1 = *reinterpret_cast<const uint32_t*>(vn);
-            qv[0] = bf16_lo(q1); qv[1] = bf16_hi(q1);
-            kv[0] = bf16_lo(k1); kv[1] = bf16_hi(k1);
-            vv[0] = bf16_lo(v1); vv[1] = bf16_hi(v1);
+            qv[2] = bf16_lo(q2.y); qv[3] = bf16_hi(q2.y);
+            kv[2] = bf16_lo(k2.y); kv[3] = bf16_hi(k2.y);
+            vv[2] = bf16_lo(v2.y); vv[3] = bf16_hi(v2.y);
         }
         float sdot = 0.f;
 #pragma unroll
@@ -897,11 +907,11 @@ __device__ __forceinline__ void row_merge(const AttnParams& p, int row, int base
         if (h == 0) {   // the token into slot s_new for the calls that follow
             const size_t s16 = (size_t)row * d.cap_o + s_new;
             if constexpr (VEC == 4) {
-                *reinterpret_cast<uint2*>(p.c.k16 + s16 * D + VEC * lane) = *reinterpret_cast<const uint2*>(kn);
-                *reinterpret_cast<uint2*>(p.c.v16 + s16 * D + VEC * lane) = *reinterpret_cast<const uint2*>(vn);
+                *reinterpret_cast<uint2*>(p.c.k16 + s16 * D + VEC * lane) = k2;
+                *reinterpret_cast<uint2*>(p.c.v16 + s16 * D + VEC * lane) = v2;
             } else {
-                *reinterpret_cast<uint32_t*>(p.c.k16 + s16 * D + VEC * lane) = *reinterpret_cast<const uint32_t*>(kn);
-                *reinterpret_cast<uint32_t*>(p.c.v16 + s16 * D + VEC * lane) = *reinterpret_cast<const uint32_t*>(vn);
+                *reinterpret_cast<uint32_t*>(p.c.k16 + s16 * D + VEC * lane) = k2.x;
+                *reinterpret_cast<uint32_t*>(p.c.v16 + s16 * D + VEC * lane) = v2.x;
             }
             if (lane == 0) {
                 p.c.pos16[s16] = p.ctx_len[b] + p.step;
@@ -964,11 +974,14 @@ __global__ void __launch_bounds__(32 * kWarps, ARKV_MIN_CTAS) decode_attn_kernel
         }
     }
 
-    // the row's ticket: every CTA of the row takes one after its partial is visible;
-    // the last one merges and moves the row's bf16 count
-    __threadfence();
+    // the row's ticket: every CTA of the row takes one after its partial is visible
+    // (the barrier, then thread 0's device-scope fence, which is cumulative over the
+    // CTA's writes ordered before it); the last one merges and moves the bf16 count
     __syncthreads();
-    if (tid == 0) sm_ticket = atomicAdd(&p.counter[row], 1u);
+    if (tid == 0) {
+        __threadfence();
+        sm_ticket = atomicAdd(&p.counter[row], 1u);
+    }
     __syncthreads();
     if (sm_ticket != (unsigned)(sh.n - 1)) return;
     __threadfence();
@@ -1100,9 +1113,13 @@ cudaError_t launch_decode_attn(AttnParams& p, cudaStream_t s) {
             resident[which][dev] = n > 0 ? n : 1;
         }
         // one wave of CTAs, at most one per 16 units (eight bf16 tiles) of the largest
-        // cache, at least one per row
+        // cache, at least one per row.  With ARKV_GRID_RESERVE, min(R, slots / 8) of the
+        // GPU's CTA slots stay out of the grid: the previous call's merging CTAs (one per
+        // row) still hold slots when this call's blocks launch, and the blocks that
+        // would wait for them start the stream late
         const long long units = (long long)d.R * (2 * ((d.cap_o + 16) / 16) + (d.cap_q + 15) / 16);
         long long P = dev < 64 ? (long long)sms[dev] * resident[which][dev] : 444;
+        if (kGridReserve) P -= (d.R < P / 8 ? d.R : P / 8);
         P = P < units / 16 ? P : units / 16;
         if (P > kMaxGrid) P = kMaxGrid;
         if (P < d.R) P = d.R;
