@@ -60,10 +60,11 @@ constexpr unsigned kFull = 0xffffffffu;
 #endif
 constexpr int kQkChains = ARKV_QK_CHAINS;   // independent QK^T accumulator chains per n-tile
 constexpr int kWarps = 4;
-#ifndef ARKV_GRID_RESERVE
-#define ARKV_GRID_RESERVE 1
+#ifndef ARKV_ROW_MULTIPLE
+#define ARKV_ROW_MULTIPLE 1
 #endif
-constexpr bool kGridReserve = ARKV_GRID_RESERVE != 0;
+constexpr bool kRowMultiple = ARKV_ROW_MULTIPLE != 0;
+
 constexpr int kSlots = 4;                  // ring slots per warp: a bf16 tile takes 2, an FP8 tile 1
 constexpr int kSpinLimit = 1 << 20;        // bounded mbarrier waits (~1 s worst case)
 constexpr int kMaxGrid = 2048;             // CTAs of one call at most (partial slots in the workspace)
@@ -171,6 +172,18 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// L2 prefetch of the 128-byte line holding `ptr`.
+__device__ __forceinline__ void prefetch_l2(const void* ptr) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr) : "memory");
+}
+
+// atomicAdd(p, 1) with acquire-release semantics at device scope.
+__device__ __forceinline__ unsigned ticket_acq_rel(unsigned* p) {
+    unsigned old;
+    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+    return old;
+}
 
 __device__ __forceinline__ void prefetch_map(const CUtensorMap* m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -635,8 +648,16 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
     for (int mt = 0; mt < KB; ++mt) oacc[mt][0] = oacc[mt][1] = oacc[mt][2] = oacc[mt][3] = 0.f;
 
     // everything above read only this layer's cache and ctx_len; q, k_new, v_new and
-    // the workspace may come from the previous kernel
-    if (p.early_start) pdl_wait();
+    // the workspace may come from the previous kernel.  Before the wait the group's
+    // queries are only prefetched to L2 (a prefetch reads nothing the kernel uses: L2
+    // stays coherent with the previous kernel's writes)
+    if (p.early_start) {
+        if (tid < 4 * D * 2 / 128 && tid / (D * 2 / 128) < d.G) {
+            const int h = tid / (D * 2 / 128), c = tid % (D * 2 / 128);
+            prefetch_l2(p.q + ((size_t)b * d.hq + gk * d.G + h) * D + 64 * c);
+        }
+        pdl_wait();
+    }
     for (int i = tid; i < 4 * D / 8; i += blockDim.x) {   // the group's queries, zero past G
         const int h = i / (D / 8), c = i - h * (D / 8);
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
@@ -974,17 +995,15 @@ __global__ void __launch_bounds__(32 * kWarps, ARKV_MIN_CTAS) decode_attn_kernel
         }
     }
 
-    // the row's ticket: every CTA of the row takes one after its partial is visible
-    // (the barrier, then thread 0's device-scope fence, which is cumulative over the
-    // CTA's writes ordered before it); the last one merges and moves the bf16 count
+    // the row's ticket: every CTA of the row takes one after its partial is written.
+    // Thread 0's acquire-release atomic is cumulative over the CTA's writes ordered
+    // before it by the barrier (release), and the barrier after it orders the last
+    // CTA's reads of the other partials after it (acquire); the last one merges and
+    // moves the bf16 count
     __syncthreads();
-    if (tid == 0) {
-        __threadfence();
-        sm_ticket = atomicAdd(&p.counter[row], 1u);
-    }
+    if (tid == 0) sm_ticket = ticket_acq_rel(&p.counter[row]);
     __syncthreads();
     if (sm_ticket != (unsigned)(sh.n - 1)) return;
-    __threadfence();
     row_merge<D>(p, row, sh.base, sh.n, append ? n16 : -1);
     if (tid == 0) {
         p.counter[row] = 0u;                                   // ready for the next call
@@ -1113,13 +1132,12 @@ cudaError_t launch_decode_attn(AttnParams& p, cudaStream_t s) {
             resident[which][dev] = n > 0 ? n : 1;
         }
         // one wave of CTAs, at most one per 16 units (eight bf16 tiles) of the largest
-        // cache, at least one per row.  With ARKV_GRID_RESERVE, min(R, slots / 8) of the
-        // GPU's CTA slots stay out of the grid: the previous call's merging CTAs (one per
-        // row) still hold slots when this call's blocks launch, and the blocks that
-        // would wait for them start the stream late
+        // cache, at least one per row.  When a multiple of R keeps at least 7/8 of the
+        // wave it is taken: rows of equal length then get equal numbers of CTAs (with 412
+        // CTAs for 32 rows, 4 rows get 12 and carry 8% more per CTA, and set the tail)
         const long long units = (long long)d.R * (2 * ((d.cap_o + 16) / 16) + (d.cap_q + 15) / 16);
         long long P = dev < 64 ? (long long)sms[dev] * resident[which][dev] : 444;
-        if (kGridReserve) P -= (d.R < P / 8 ? d.R : P / 8);
+        if (kRowMultiple && d.R <= P && (P / d.R) * d.R * 8 >= P * 7) P = (P / d.R) * d.R;
         P = P < units / 16 ? P : units / 16;
         if (P > kMaxGrid) P = kMaxGrid;
         if (P < d.R) P = d.R;
