@@ -88,3 +88,39 @@ def test_noalloc_rejects_layers_beyond_its_scratch(cuda):
                                    check=False)
     assert rc == abi.ARKV_EINVAL
     assert "scratch" in abi.arkv_last_error_string()
+
+
+def test_noalloc_reassign_in_a_cuda_graph(cuda):
+    """The entry point's stated use: captured into a CUDA graph (no allocation is
+    possible there) and replayed, it leaves the cache that arkv_reassign leaves."""
+    build()
+    wl = SMALL_D128_G3
+    r = wl.r_bar
+    t_re = wl.reassign_interval - 1
+    cap_o, cap_q = H.capacities(wl, r, wl.n_ctx + wl.reassign_interval)
+    a = H.DeviceLayer(wl, cap_o, cap_q, cuda)
+    pre = inputs.layer_prefill(wl, 0)
+    to = lambda bits: H.bits_to_bf16_tensor(bits, cuda)
+    ctx = torch.from_numpy(pre["ctx_len"]).to(cuda)
+    a.prefill(to(pre["k"]), to(pre["v"]), to(pre["q_obs"]), ctx, r=r)
+    o = torch.zeros((wl.batch, wl.hq, wl.head_dim), dtype=torch.float32, device=cuda)
+    for t in range(t_re + 1):
+        d = inputs.decode_inputs(wl, 0, t)
+        a.decode(t, to(d["q"]), to(d["k_new"]), to(d["v_new"]), ctx, o)
+        a.score(t, ctx)
+    b_cache = _clone_cache(a.cache, a.cfg, cuda)
+    warm = _clone_cache(a.cache, a.cfg, cuda)
+    # the first call looks the scratch address up, which a capture does not allow
+    abi.arkv_reassign_noalloc(a.cfg, t_re, r, ctx.data_ptr(), warm.c, None, stream_ptr())
+    torch.cuda.synchronize()
+    td_b = torch.full_like(a.tier_dbg, 255)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        abi.arkv_reassign_noalloc(a.cfg, t_re, r, ctx.data_ptr(), b_cache.c, td_b.data_ptr(), stream_ptr())
+    g.replay()
+    a.reassign(t_re, r, ctx)
+    torch.cuda.synchronize()
+    assert torch.equal(a.tier_dbg, td_b)
+    assert int((td_b != 255).sum()) > 0
+    _same_cache(a.cache, b_cache)
+    del g
