@@ -6,9 +6,9 @@
 // proportion to their lengths; each CTA takes the same fraction of its row's bf16
 // tiles and of its FP8 tiles (16 tokens each), bf16 tiles first.  Its 4 warps take
 // the tiles round robin, each through its own ring of 4 shared-memory slots (a bf16
-// tile takes two, K then V; an FP8 tile one) filled by TMA tensor loads (16 rows per
-// box, 128-byte swizzle; 64-byte for FP8 rows of 64 bytes) completing on per-slot
-// mbarriers (waits are bounded).
+// tile takes two, K and V, each freed as soon as it is read; an FP8 tile one) filled
+// by TMA tensor loads (16 rows per box, 128-byte swizzle; 64-byte for FP8 rows of 64
+// bytes) completing on per-slot mbarriers (waits are bounded).
 //
 // Tile math on the warp-level tensor cores (m16n8k16).  QK^T with the queries as
 // the M rows: rows 0..3 and 4..7 both hold the group's heads (zero past G), rows
@@ -262,9 +262,9 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // ------------------------------------------------------------------ per-lane addresses
-// Shared-memory byte offsets (from a tile's first ring slot) of the fragment loads
-// of one lane; index j = 0..3 selects a 32-byte column pair (two 16-byte chunks) of
-// the row.  A bf16 tile holds K in its first slot and V in the next; an FP8 tile
+// Shared-memory byte offsets of the fragment loads of one lane, K from the tile's K
+// slot and V from its V slot; index j = 0..3 selects a 32-byte column pair (two
+// 16-byte chunks) of the row.  A bf16 tile has a K slot and a V slot; an FP8 tile
 // holds K and V (16 x D bytes each) in one slot.  Fragment conventions of
 // m16n8k16: lane = 4 g + t.
 template <int D, bool FP8>
@@ -272,7 +272,7 @@ struct LaneOffsets {
     uint32_t k[4], v[4];
     __device__ __forceinline__ LaneOffsets() {
         const int lane = threadIdx.x & 31, m = lane >> 3;
-        constexpr int VOFF = FP8 ? 16 * D : Smem<D>::kSlot;
+        constexpr int VOFF = FP8 ? 16 * D : 0;   // a bf16 tile's V has a slot of its own
         if constexpr (!FP8) {
             // K, ldmatrix.x4: matrix m = (tokens 8 (m >> 1) .., chunk 2j + (m & 1)) -> the
             // B fragments (b0, b1) of n-tiles 0 and 1 for k block j (16 dims = 2 chunks).
@@ -315,11 +315,15 @@ struct RowState {
 // heads, rows 8..15 are zero).  skv/svv: FP8 scales of this lane's tokens 2t, 2t+1,
 // 8+2t, 9+2t (unused for bf16); vnorm: the warp's V-scale normaliser.  hv: this
 // lane's head (g & 3) is real; lo: this lane supplies the low parts of P (g >= 4).
-template <int D, bool FP8, int FMT>
-__device__ __forceinline__ void attend_tile(uint32_t st, const LaneOffsets<D, FP8>& off, int t0, int seg_end,
-                                            bool hv, bool lo, float c2, const float (&skv)[4], const float (&svv)[4],
-                                            float vnorm, float* logit_head, const uint32_t (&qa)[D / 16][2],
-                                            RowState& rs, float (&oacc)[D / 16][4]) {
+// `sv` is the shared address of the V tile (the K slot's address for FP8 tiles); `mid`
+// runs between QK^T and PV (it frees the K slot and waits for the V slot of a bf16
+// tile) and returns false if V did not arrive, in which case PV is skipped.
+template <int D, bool FP8, int FMT, typename Mid>
+__device__ __forceinline__ void attend_tile(uint32_t st, uint32_t sv, const LaneOffsets<D, FP8>& off, int t0,
+                                            int seg_end, bool hv, bool lo, float c2, const float (&skv)[4],
+                                            const float (&svv)[4], float vnorm, float* logit_head,
+                                            const uint32_t (&qa)[D / 16][2], RowState& rs,
+                                            float (&oacc)[D / 16][4], Mid&& mid) {
     constexpr int KB = D / 16;   // k blocks of QK^T, m-tiles of PV
     const int lane = threadIdx.x & 31;
     const int t = lane & 3;
@@ -433,11 +437,12 @@ __device__ __forceinline__ void attend_tile(uint32_t st, const LaneOffsets<D, FP
         m0 = (tA < seg_end ? 0xffffu : 0u) | (tA + 1 < seg_end ? 0xffff0000u : 0u);
         m1 = (tB < seg_end ? 0xffffu : 0u) | (tB + 1 < seg_end ? 0xffff0000u : 0u);
     }
+    if (!mid()) return;
     if constexpr (!FP8) {
 #pragma unroll
         for (int mt = 0; mt < KB; ++mt) {
             uint32_t af[4];   // A fragment of V^T for dims 16 mt .. 16 mt + 15
-            ldsm_x4_trans(af, st + off.v[mt & 3] + (mt >> 2) * 2048);
+            ldsm_x4_trans(af, sv + off.v[mt & 3] + (mt >> 2) * 2048);
             if (partial) { af[0] &= m0; af[1] &= m0; af[2] &= m1; af[3] &= m1; }
             mma16816<false>(oacc[mt], af[0], af[1], af[2], af[3], b0, b1);
         }
@@ -445,7 +450,7 @@ __device__ __forceinline__ void attend_tile(uint32_t st, const LaneOffsets<D, FP
 #pragma unroll
         for (int j = 0; j < KB / 2; ++j) {
             uint32_t r[4];   // chunk 2j: dims +g (r0), +8+g (r1); chunk 2j+1: r2, r3
-            ldsm_b8_x2_trans(r, st + off.v[j]);
+            ldsm_b8_x2_trans(r, sv + off.v[j]);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t a0, a2, a1, a3;
@@ -600,24 +605,23 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
         const int li = warp + kWarps * i;
         return li < L16 ? (a16 + li) << 1 : ((a8 + li - L16) << 1) | 1;
     };
-    // producer state (every lane keeps it; lane 0 issues the tensor loads)
-    int iss = 0, ipos = 0, free_slots = kSlots;
+    // producer state (every lane keeps it; lane 0 issues the tensor loads).  The ring
+    // holds entries, one slot each: a bf16 tile is two (its K, then its V), so its K slot
+    // is refilled as soon as QK^T has read it; an FP8 tile is one (K and V)
+    int iss = 0, half = 0, ipos = 0, free_slots = kSlots, ient = 0;
     auto try_issue = [&]() {
-        while (iss < nt) {
+        while (iss < nt && free_slots > 0) {
             const int enc = enc_of(iss);
             const bool f8 = enc & 1;
-            const int jt = enc >> 1, sz = f8 ? 1 : 2;
-            if (sz > free_slots) break;
+            const int jt = enc >> 1;
             const uint32_t dst = ring + ipos * SLOT, bar = bars + 8 * ipos;
             if (lane == 0) {
                 if (!f8) {
                     const int y = row * d.cap_o + 16 * jt;
-                    mbar_expect_tx(bar, 2 * SLOT);
+                    const CUtensorMap* m = half == 0 ? &p.tm_k16 : &p.tm_v16;
+                    mbar_expect_tx(bar, SLOT);
 #pragma unroll
-                    for (int bx = 0; bx < D * 2 / 128; ++bx) {
-                        tma_load_2d(dst + bx * 2048, &p.tm_k16, bx * 64, y, bar);
-                        tma_load_2d(dst + SLOT + bx * 2048, &p.tm_v16, bx * 64, y, bar);
-                    }
+                    for (int bx = 0; bx < D * 2 / 128; ++bx) tma_load_2d(dst + bx * 2048, m, bx * 64, y, bar);
                 } else {
                     const int y = row * d.cap_q + 16 * jt;
                     mbar_expect_tx(bar, 2 * 16 * D);
@@ -630,11 +634,17 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
                 cp_async4(sc_base + (ipos * 32 + lane) * 4,
                           (lane < 16 ? p.c.sk : p.c.sv) + (size_t)row * d.cap_q + tok);
             }
-            cp_async_commit();
+            cp_async_commit();   // one group per entry
             sm_tq[ipos] = enc;
-            ipos = (ipos + sz) & (kSlots - 1);
-            free_slots -= sz;
-            ++iss;
+            ipos = (ipos + 1) & (kSlots - 1);
+            --free_slots;
+            ++ient;
+            if (f8 || half == 1) {
+                ++iss;
+                half = 0;
+            } else {
+                half = 1;
+            }
         }
     };
     try_issue();
@@ -666,11 +676,11 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
     }
     __syncthreads();
 
-    int pos = 0;          // ring slot of the next tile to consume
+    int pos = 0;          // ring slot of the next entry to consume
     uint32_t ph = 0;      // parity of every slot's next phase
-    int cons = 0;         // tiles consumed
+    int cent = 0;         // entries consumed
     bool aborted = false;
-    auto wait_tile = [&]() -> bool {
+    auto wait_entry = [&]() -> bool {
         if (mbar_wait(bars + 8 * pos, (ph >> pos) & 1u)) return true;
         // a copy did not land in time: flag it, give every copy this warp has in flight
         // (this one included) a last bounded chance to land, and leave the ring alone
@@ -679,18 +689,18 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
             atomicExch(sm_abort, 1);
         }
         uint32_t q = ph;
-        for (int j = cons, sp = pos; j < iss; ++j) {
+        for (int j = cent, sp = pos; j < ient; ++j) {
             mbar_wait(bars + 8 * sp, (q >> sp) & 1u);
             q ^= 1u << sp;
-            sp = (sp + ((sm_tq[sp] & 1) ? 1 : 2)) & (kSlots - 1);
+            sp = (sp + 1) & (kSlots - 1);
         }
         return false;
     };
-    auto release = [&](int sz) {
+    auto release = [&]() {   // frees the entry at pos
         ph ^= 1u << pos;
-        pos = (pos + sz) & (kSlots - 1);
-        free_slots += sz;
-        ++cons;
+        pos = (pos + 1) & (kSlots - 1);
+        ++free_slots;
+        ++cent;
         __syncwarp();
         try_issue();
     };
@@ -705,10 +715,17 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
         const float one[4] = {1.f, 1.f, 1.f, 1.f};
         for (int i = 0; i < nt16; ++i) {
             const int t0 = 16 * (sm_tq[pos] >> 1);
-            if (!wait_tile()) { aborted = true; break; }
-            attend_tile<D, false, FMT>(ring + pos * SLOT, off, t0, n16, hv, lo, c2, one, one, 1.f, logit_head, qa,
-                                       rs, oacc);
-            release(2);
+            if (!wait_entry()) { aborted = true; break; }
+            const uint32_t sk = ring + pos * SLOT, sv = ring + ((pos + 1) & (kSlots - 1)) * SLOT;
+            bool v_ok = true;
+            attend_tile<D, false, FMT>(sk, sv, off, t0, n16, hv, lo, c2, one, one, 1.f, logit_head, qa, rs, oacc,
+                                       [&]() {   // K is read: free its slot, then wait for V
+                                           release();
+                                           v_ok = wait_entry();
+                                           return v_ok;
+                                       });
+            if (!v_ok) { aborted = true; break; }
+            release();
         }
     }
     // ---- FP8 tiles
@@ -718,9 +735,9 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
         float* logit_head = p.logit8 + ((size_t)row * 4 + (hv ? hd : 0)) * p.lstride_q;
         for (int i = nt16; i < nt; ++i) {
             const int t0 = 16 * (sm_tq[pos] >> 1);
-            if (!wait_tile()) { aborted = true; break; }
-            // this tile's scale group (the groups of later tiles may still be in flight)
-            switch (iss - cons - 1) {
+            if (!wait_entry()) { aborted = true; break; }
+            // this tile's scale group (the groups of later entries may still be in flight)
+            switch (ient - cent - 1) {
                 case 0: cp_async_wait<0>(); break;
                 case 1: cp_async_wait<1>(); break;
                 case 2: cp_async_wait<2>(); break;
@@ -750,9 +767,10 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
                 vnorm = vn;
                 vcur = m;
             }
-            attend_tile<D, true, FMT>(ring + pos * SLOT, off, t0, n8, hv, lo, c2, skv, svv, vnorm, logit_head, qa,
-                                      rs, oacc);
-            release(1);
+            const uint32_t st = ring + pos * SLOT;
+            attend_tile<D, true, FMT>(st, st, off, t0, n8, hv, lo, c2, skv, svv, vnorm, logit_head, qa, rs, oacc,
+                                      []() { return true; });
+            release();
         }
     }
     cp_async_wait<0>();
