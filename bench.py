@@ -6,8 +6,9 @@
 A step is one decode step of the whole attention stack: for every layer, append +
 mixed-precision attention (arkv_decode_attn), score update (arkv_score_update),
 and the tier reassignment (arkv_reassign) on every reassign_interval-th step.  The
-score update and reassignment of a layer run on a second stream, beside the next
-layers' attention; the layer's next attention call waits for them.
+score update and reassignment of a layer run on a side stream (layers dealt round
+robin over --streams - 1 of them), beside the next layers' attention; the layer's next
+attention call waits for them.
 Each GPU runs its own replica of the workload (independent sequences; no
 collective on the data path), so `value` is the tokens/s of all ranks together
 ("scaling": "weak").  Inputs are synthetic and seeded; each step streams the whole
@@ -45,9 +46,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--streams", type=int, default=2, choices=[1, 2],
-                    help="2: score updates and reassignments on a second stream beside the next layers' "
-                         "attention; 1: everything on one stream")
+    ap.add_argument("--streams", type=int, default=5,
+                    help="S >= 2: score updates and reassignments on S - 1 side streams (layer l on side "
+                         "stream l mod (S - 1)) beside the next layers' attention; 1: everything on one stream")
     ap.add_argument("--no-early-start", action="store_true",
                     help="launch every attention call with early_start = 0 (it waits for the previous "
                          "kernel before reading its cache)")
@@ -320,13 +321,14 @@ def run_reference(args, wl, rank):
     print(json.dumps(line), flush=True)
 
 
-def config_of(wl, streams=2, early=None):
+def config_of(wl, streams=5, early=None):
     return {"workload": wl.name, "layers": wl.layers, "batch": wl.batch, "hq": wl.hq, "hkv": wl.hkv,
             "head_dim": wl.head_dim, "n_ctx": wl.n_ctx, "n_ctx_min": wl.n_ctx_min,
             "budget_frac": wl.budget_frac, "oq_ratio": wl.oq_ratio if wl.oq_ratio is not None
             else f"per layer from prefill stats (r_bar {wl.r_bar})", "window": wl.window,
             "gamma": wl.gamma, "reassign_interval": wl.reassign_interval, "quant_format": wl.quant_format,
-            "streams": "score update and reassignment on a second stream" if streams == 2 else "one stream",
+            "streams": (f"score update and reassignment on {streams - 1} side stream(s), layers round robin"
+                        if streams >= 2 else "one stream"),
             "l2": "no flush: every step streams the whole compressed cache, far above L2",
             "early_start": (wl.layers >= 3) if early is None else bool(early)}
 
@@ -403,10 +405,12 @@ def run_arkv(args, wl, rank, world, local_rank):
     o = torch.zeros((L, B, Hq, D), dtype=torch.float32, device=dev)
     launches = {"n": 0}
 
-    # The score update and reassignment of layer l run on a side stream: the next
-    # layer's attention does not wait for them (in a model, the next layer's query
-    # needs only this layer's output).  The next call on layer l's cache waits for them.
-    side = torch.cuda.Stream(device=dev) if args.streams == 2 else None
+    # The score update and reassignment of layer l run on side stream l mod (S - 1): the
+    # next layer's attention does not wait for them (in a model, the next layer's query
+    # needs only this layer's output), and the reassignments of a reassignment step, one
+    # row per CTA, run side by side on several streams instead of one after another.
+    # The next call on layer l's cache waits for them.
+    sides = [torch.cuda.Stream(device=dev) for _ in range(max(args.streams - 1, 0))]
     pending = {}                                             # layer -> event after its side work
 
     def settle(l):
@@ -432,6 +436,7 @@ def run_arkv(args, wl, rank, world, local_rank):
                              o[l].data_ptr(), x["ws_d"].ptr, x["ws_d"].nbytes, main.cuda_stream)
         if ev is not None:
             ev[1].record(main)
+        side = sides[l % len(sides)] if sides else None
         aux = side if side is not None else main
         if side is not None:
             attended = torch.cuda.Event()

@@ -268,6 +268,8 @@ __device__ __forceinline__ float warp_quantize_row(const uint16_t* src, uint8_t*
 }
 
 // ------------------------------------------------------------------ reassignment
+constexpr int kKeyBatch = 8;   // slots per thread whose loads are in flight together (key build)
+
 // Slot outcomes, frozen before any data moves.
 constexpr uint64_t kStayBf16 = 0, kDemote = 1, kEvict = 2, kStayFp8 = 3;
 
@@ -293,20 +295,34 @@ __global__ void __launch_bounds__(kRowThreads) reassign_kernel(const ReassignPar
 
     auto pos_of = [&](int i) -> int { return i < n16 ? p.c.pos16[b16 + i] : p.c.pos8[b8 + (i - n16)]; };
 
-    // keys: 0 for window tokens (never candidates), order-preserving map of S otherwise
+    // keys: 0 for window tokens (never candidates), order-preserving map of S otherwise.
+    // kKeyBatch slots per thread at a time, all their loads issued before any of them is
+    // used, so that the row's ~n / 1024 memory latencies per thread overlap
     int ncand = 0;
-    for (int i = tid; i < n; i += blockDim.x) {
-        const bool bf = i < n16;
-        const size_t sl = bf ? b16 + i : b8 + (i - n16);
-        const int pos = bf ? p.c.pos16[sl] : p.c.pos8[sl];
-        uint64_t key = 0;
-        if (!bf || pos < winlo) {
-            const double mu = bf ? p.c.mu16[sl] : p.c.mu8[sl];
-            const double m2 = bf ? p.c.m2_16[sl] : p.c.m2_8[sl];
-            key = double_key(score_f64(mu, m2, obs_count_after(pos, n0, p.step, d.n_obs), d.gamma));
-            ++ncand;
+    for (int base = 0; base < n; base += kKeyBatch * (int)blockDim.x) {
+        int pos[kKeyBatch];
+        double mu[kKeyBatch], m2[kKeyBatch];
+#pragma unroll
+        for (int u = 0; u < kKeyBatch; ++u) {
+            const int i = base + u * (int)blockDim.x + tid;
+            const bool bf = i < n16;
+            const size_t sl = bf ? b16 + i : b8 + (i - n16);
+            const bool in = i < n;
+            pos[u] = in ? (bf ? p.c.pos16[sl] : p.c.pos8[sl]) : 0;
+            mu[u] = in ? (bf ? p.c.mu16[sl] : p.c.mu8[sl]) : 0.0;
+            m2[u] = in ? (bf ? p.c.m2_16[sl] : p.c.m2_8[sl]) : 0.0;
         }
-        keys[i] = key;
+#pragma unroll
+        for (int u = 0; u < kKeyBatch; ++u) {
+            const int i = base + u * (int)blockDim.x + tid;
+            if (i >= n) break;
+            uint64_t key = 0;
+            if (i >= n16 || pos[u] < winlo) {
+                key = double_key(score_f64(mu[u], m2[u], obs_count_after(pos[u], n0, p.step, d.n_obs), d.gamma));
+                ++ncand;
+            }
+            keys[i] = key;
+        }
     }
     ncand = block_sum(ncand, sh);
     if (tid == 0) {
