@@ -224,6 +224,19 @@ int arkv_reassign(const arkv_cfg *cfg, int32_t step, float r, const int32_t *ctx
  * out[i] = code(x[i]), n elements. */
 int arkv_fp8_encode(int32_t format, const float *x, uint8_t *out, size_t n, arkv_stream_t stream);
 
+/* Host <-> device transfer for the decode loop's inputs and outputs, done by a
+ * device kernel instead of the copy engine: copies `bytes` from src to dst, either of
+ * which may be device memory or page-locked host memory (cudaHostAlloc /
+ * cudaHostRegister; the device reads and writes it over the bus under unified
+ * addressing).  Captured into a CUDA graph it is a kernel node, which keeps
+ * programmatic dependent launches and the graph's concurrent branches intact around
+ * it, where a copy-engine node between kernels costs a synchronisation.
+ * bytes a multiple of 16 and both addresses 16-byte aligned, else ARKV_EINVAL.
+ * Pointers the device cannot address (pageable host memory) are rejected with
+ * ARKV_EINVAL before any launch (cudaPointerGetAttributes); make the first call on
+ * a buffer outside any stream capture.  The buffers must not overlap. */
+int arkv_copy_async(void *dst, const void *src, size_t bytes, arkv_stream_t stream);
+
 /* Allocation-free tier reassignment.  The paper has no counterpart: this is an
  * interface for callers that cannot allocate device memory when they reassign --
  * code running while a CUDA graph is captured (cudaMalloc is not a stream

@@ -57,6 +57,7 @@ _SIG = {
     "arkv_reassign": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_float, _P, _P, _P, _P,
                                      ctypes.c_size_t, _P]),
     "arkv_fp8_encode": (ctypes.c_int, [ctypes.c_int32, _P, _P, ctypes.c_size_t, _P]),
+    "arkv_copy_async": (ctypes.c_int, [_P, _P, ctypes.c_size_t, _P]),
     "arkv_reassign_noalloc": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_float, _P, _P, _P, _P]),
     "arkv_last_error_string": (ctypes.c_char_p, []),
 }
@@ -144,6 +145,11 @@ def arkv_reassign_noalloc(cfg, step, r, ctx_len, cache, tier_dbg, stream, check=
     """arkv_reassign without a workspace (scratch in the library's static device array)."""
     rc = lib().arkv_reassign_noalloc(_ref(cfg), step, r, ctx_len, _ref(cache), tier_dbg, stream)
     return _check("arkv_reassign_noalloc", rc) if check else rc
+
+
+def arkv_copy_async(dst, src, nbytes, stream, check=True) -> int:
+    rc = lib().arkv_copy_async(dst, src, nbytes, stream)
+    return _check("arkv_copy_async", rc) if check else rc
 
 
 def arkv_fp8_encode(fmt, x, out, n, stream, check=True) -> int:

@@ -251,6 +251,31 @@ int arkv_reassign(const arkv_cfg* cfg, int32_t step, float r, const int32_t* ctx
     return e == cudaSuccess ? ARKV_OK : cuda_fail(e, "arkv_reassign");
 }
 
+// True if the device can address ptr: device memory, or page-locked host memory mapped
+// into the unified address space (its device pointer is the host pointer).
+static bool device_addressable(const void* ptr) {
+    cudaPointerAttributes at{};
+    if (cudaPointerGetAttributes(&at, ptr) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) return true;
+    return at.type == cudaMemoryTypeHost && at.devicePointer == ptr;
+}
+
+int arkv_copy_async(void* dst, const void* src, size_t bytes, arkv_stream_t stream) {
+    if (bytes == 0) return ARKV_OK;
+    if (!dst || !src) return fail(ARKV_EINVAL, "%s: null argument", "arkv_copy_async");
+    if ((bytes & 15) || !aligned(dst, 16) || !aligned(src, 16))
+        return fail(ARKV_EINVAL, "%s: bytes and both addresses must be multiples of 16", "arkv_copy_async");
+    const uintptr_t d0 = (uintptr_t)dst, s0 = (uintptr_t)src;
+    if (d0 < s0 + bytes && s0 < d0 + bytes) return fail(ARKV_EINVAL, "%s: the buffers overlap", "arkv_copy_async");
+    if (!device_addressable(dst) || !device_addressable(src))
+        return fail(ARKV_EINVAL, "%s: a buffer is not device-addressable (pageable host memory?)", "arkv_copy_async");
+    const cudaError_t e = arkv::launch_copy16(dst, src, bytes, (cudaStream_t)stream);
+    return e == cudaSuccess ? ARKV_OK : cuda_fail(e, "arkv_copy_async");
+}
+
 int arkv_fp8_encode(int32_t format, const float* x, uint8_t* out, size_t n, arkv_stream_t stream) {
     if (format != ARKV_FMT_E4M3 && format != ARKV_FMT_E5M2)
         return fail(ARKV_EINVAL, "%s: unknown format", "arkv_fp8_encode");

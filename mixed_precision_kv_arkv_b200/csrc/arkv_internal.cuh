@@ -165,6 +165,7 @@ DecodeWs decode_ws_layout(const LayerDims& d);
 
 cudaError_t launch_decode_attn(AttnParams& p, cudaStream_t s);   // fills the tensor maps
 cudaError_t launch_score_update(const ScoreParams& p, cudaStream_t s);
+cudaError_t launch_copy16(void* dst, const void* src, size_t bytes, cudaStream_t s);   // bytes % 16 == 0
 
 struct ReassignParams {
     LayerDims d;

@@ -103,3 +103,15 @@ def test_null_cache_buffers_and_small_workspace_rejected(lib):
     small = cfg(cap_bf16=10, cap_fp8=10)
     assert abi.arkv_quantize_pack(small, 0.5, p, p, 2048, p, p, p, cache, None, p, 1 << 30, None,
                                   check=False) == abi.ARKV_ECAPACITY
+
+
+def test_copy_async_rejects_bad_arguments_before_any_launch(lib):
+    """Alignment, size and overlap are checked on the host, before the pointers are
+    even inspected (no GPU needed)."""
+    a, b = ctypes.c_void_p(4096), ctypes.c_void_p(1 << 20)
+    assert abi.arkv_copy_async(a, b, 0, None) == abi.ARKV_OK           # nothing to copy
+    assert abi.arkv_copy_async(None, b, 16, None, check=False) == abi.ARKV_EINVAL
+    assert abi.arkv_copy_async(a, b, 24, None, check=False) == abi.ARKV_EINVAL                # size % 16
+    assert abi.arkv_copy_async(ctypes.c_void_p(4104), b, 32, None, check=False) == abi.ARKV_EINVAL   # dst % 16
+    assert abi.arkv_copy_async(a, ctypes.c_void_p(4096 + 16), 64, None, check=False) == abi.ARKV_EINVAL  # overlap
+    assert "arkv_copy_async" in abi.arkv_last_error_string()
