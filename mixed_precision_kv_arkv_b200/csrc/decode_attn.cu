@@ -854,10 +854,12 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
 // dropped) enters here as one more term: its logit q . k_new (float32 products of
 // the bf16 values, summed over the warp), its weight exp((q.k - M')/sqrt(D)) and
 // its value v_new; its raw logit goes to the workspace with the others, and the
-// token is stored in slot s_new for later calls (no tensor load of this call reads
-// that slot).  Publishes (M, L) for the score update.
+// token is stored in slot s_new at position pos_new for later calls (no tensor load
+// of this call reads that slot).  Publishes (M, L) for the score update.  Every
+// global load of the merge is issued before its arithmetic, so that the merge ends in
+// stores only.
 template <int D>
-__device__ __forceinline__ void row_merge(const AttnParams& p, int row, int base, int n, int s_new) {
+__device__ __forceinline__ void row_merge(const AttnParams& p, int row, int base, int n, int s_new, int pos_new) {
     constexpr int VEC = D / 32;
     constexpr int kBatch = 16;
     const LayerDims& d = p.d;
@@ -953,7 +955,7 @@ __device__ __forceinline__ void row_merge(const AttnParams& p, int row, int base
                 *reinterpret_cast<uint32_t*>(p.c.v16 + s16 * D + VEC * lane) = v2.x;
             }
             if (lane == 0) {
-                p.c.pos16[s16] = p.ctx_len[b] + p.step;
+                p.c.pos16[s16] = pos_new;
                 p.c.mu16[s16] = 0.0;
                 p.c.m2_16[s16] = 0.0;
             }
@@ -989,6 +991,7 @@ __global__ void __launch_bounds__(32 * kWarps, ARKV_MIN_CTAS) decode_attn_kernel
     const int n16 = min(max(sh.n16, 0), d.cap_o);   // counts are clamped to the
     const int n8 = min(max(sh.n8, 0), d.cap_q);      // capacities before any use
     const bool append = n16 < d.cap_o;               // the new token goes to slot n16
+    const int pos_new = p.ctx_len[row / d.hkv] + p.step;   // at this position (read at entry)
     // this CTA's share of the row: the same fraction of each segment's 16-token tiles,
     // so that every CTA of the row has the same mix of bf16 and FP8 work
     const int T16 = (n16 + 15) / 16, T8 = (n8 + 15) / 16;
@@ -1022,7 +1025,7 @@ __global__ void __launch_bounds__(32 * kWarps, ARKV_MIN_CTAS) decode_attn_kernel
     if (tid == 0) sm_ticket = ticket_acq_rel(&p.counter[row]);
     __syncthreads();
     if (sm_ticket != (unsigned)(sh.n - 1)) return;
-    row_merge<D>(p, row, sh.base, sh.n, append ? n16 : -1);
+    row_merge<D>(p, row, sh.base, sh.n, append ? n16 : -1, pos_new);
     if (tid == 0) {
         p.counter[row] = 0u;                                   // ready for the next call
         if (append) p.c.n_bf16[row] = n16 + 1;
