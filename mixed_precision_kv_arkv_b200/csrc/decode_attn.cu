@@ -56,9 +56,9 @@ constexpr unsigned kFull = 0xffffffffu;
 #define ARKV_MIN_CTAS 3
 #endif
 #ifndef ARKV_QK_CHAINS
-#define ARKV_QK_CHAINS 1
+#define ARKV_QK_CHAINS 2
 #endif
-constexpr int kQkChains = ARKV_QK_CHAINS;   // independent QK^T accumulator chains per n-tile
+constexpr int kQkChains = ARKV_QK_CHAINS;   // independent QK^T accumulator chains per tile
 constexpr int kWarps = 4;
 #ifndef ARKV_ROW_MULTIPLE
 #define ARKV_ROW_MULTIPLE 1
@@ -228,6 +228,15 @@ __device__ __forceinline__ void ldsm_b8_x2_trans(uint32_t (&r)[4], uint32_t addr
                  : "r"(addr));
 }
 
+// Transpose of an 8 x 8 matrix of 16-bit elements held one row pair per lane (lane
+// 4 r + c holds row r, columns 2c, 2c + 1): afterwards lane 4 r + c holds row r of
+// the transpose, i.e. column r of the input at rows 2c, 2c + 1.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+    uint32_t d;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+    return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -305,137 +314,154 @@ struct LaneOffsets {
 
 // ------------------------------------------------------------------ one tile
 struct RowState {
-    float m;     // reference maximum of this lane's head (raw logit units)
-    float l;     // this lane's share of the head's sum of probabilities
+    float m[2];   // reference maxima of this lane's two heads (raw logit units)
+    float l[2];   // this lane's share of their sums of probabilities
 };
 
 // One 16-token tile (tokens t0 .. t0+15 of a segment ending at seg_end) held at
-// shared address `st` (its first ring slot).  qa: the A fragments of the
-// queries (a0, a2 of every k block: rows 0..3 and 4..7 both hold the group's
-// heads, rows 8..15 are zero).  skv/svv: FP8 scales of this lane's tokens 2t, 2t+1,
-// 8+2t, 9+2t (unused for bf16); vnorm: the warp's V-scale normaliser.  hv: this
-// lane's head (g & 3) is real; lo: this lane supplies the low parts of P (g >= 4).
-// `sv` is the shared address of the V tile (the K slot's address for FP8 tiles); `mid`
-// runs between QK^T and PV (it frees the K slot and waits for the V slot of a bf16
-// tile) and returns false if V did not arrive, in which case PV is skipped.
+// shared address `st` (its first ring slot).
+//
+// S^T = K Q^T on m16n8k16: K is the A operand (16 tokens x 16 dims per k block, the
+// same ldmatrix loads that would give it as a B operand, in another register order),
+// and the queries are the B operand (qa: column n = head n & 3, so columns 4..7 repeat
+// the group).  Lane (g, t) then holds the logits of tokens g and g + 8 for columns 2t
+// and 2t + 1: heads 2t, 2t + 1 for t < 2, and the same heads again for t >= 2, whose
+// lanes supply the low parts of P.  P (16 tokens x 8 columns [hi | lo], 16-bit) is
+// taken to the B fragment of O^T += V^T P by two register transposes (movmatrix).
+// The accumulator columns of a lane are its own two heads, so a change of the
+// softmax reference rescales them without any exchange between lanes.
+//
+// skv/svv: FP8 scales of tokens g and g + 8 (unused for bf16); vnorm: the warp's
+// V-scale normaliser.  hv0/hv1: the lane's heads are real; lo: the lane supplies low
+// parts (t >= 2).  logit_row: the row's raw logits [head][lstride].  `sv` is the
+// shared address of the V tile (the K slot's address for FP8 tiles); `mid` runs
+// between QK^T and PV (it frees the K slot and waits for the V slot of a bf16 tile)
+// and returns false if V did not arrive, in which case PV is skipped.
 template <int D, bool FP8, int FMT, typename Mid>
 __device__ __forceinline__ void attend_tile(uint32_t st, uint32_t sv, const LaneOffsets<D, FP8>& off, int t0,
-                                            int seg_end, bool hv, bool lo, float c2, const float (&skv)[4],
-                                            const float (&svv)[4], float vnorm, float* logit_head,
-                                            const uint32_t (&qa)[D / 16][2], RowState& rs,
-                                            float (&oacc)[D / 16][4], Mid&& mid) {
+                                            int seg_end, bool hv0, bool hv1, bool lo, float c2,
+                                            const float (&skv)[2], const float (&svv)[2], float vnorm,
+                                            float* logit_row, int lstride, const uint32_t (&qa)[D / 16][2],
+                                            RowState& rs, float (&oacc)[D / 16][4], Mid&& mid) {
     constexpr int KB = D / 16;   // k blocks of QK^T, m-tiles of PV
+    constexpr int C = kQkChains;
     const int lane = threadIdx.x & 31;
-    const int t = lane & 3;
+    const int g = lane >> 2, t = lane & 3;
 
-    // ---- S = Qx K^T: n-tile 0 (tokens 0..7) and n-tile 1 (tokens 8..15), kQkChains
-    // independent accumulator chains per n-tile (k blocks dealt round robin)
-    float sa[2][kQkChains][4];
+    // ---- S^T = K Q^T, C independent accumulator chains (k blocks dealt round robin);
+    // element e: (token g, column 2t), (g, 2t + 1), (g + 8, 2t), (g + 8, 2t + 1)
+    float sa[C][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int c = 0; c < kQkChains; ++c) sa[nt][c][0] = sa[nt][c][1] = sa[nt][c][2] = sa[nt][c][3] = 0.f;
+    for (int c = 0; c < C; ++c) sa[c][0] = sa[c][1] = sa[c][2] = sa[c][3] = 0.f;
     if constexpr (!FP8) {
+        // ldmatrix.x4 of block kk: (tokens 0-7, dims 2t..), (tokens 0-7, dims 8+2t..),
+        // (tokens 8-15, dims 2t..), (tokens 8-15, dims 8+2t..) = A fragment a0, a2, a1, a3
 #pragma unroll
         for (int kk = 0; kk < KB; ++kk) {
-            uint32_t b[4];   // (b0, b1) of n-tile 0, then of n-tile 1
-            ldsm_x4(b, st + off.k[kk & 3] + (kk >> 2) * 2048);
-            mma16816<false>(sa[0][kk % kQkChains], qa[kk][0], 0u, qa[kk][1], 0u, b[0], b[1]);
-            mma16816<false>(sa[1][kk % kQkChains], qa[kk][0], 0u, qa[kk][1], 0u, b[2], b[3]);
+            uint32_t a[4];
+            ldsm_x4(a, st + off.k[kk & 3] + (kk >> 2) * 2048);
+            mma16816<false>(sa[kk % C], a[0], a[2], a[1], a[3], qa[kk][0], qa[kk][1]);
         }
     } else {
+        // words: (token g, block 2j), (g, 2j + 1), (g + 8, 2j), (g + 8, 2j + 1), each four
+        // codes = dims 4t..4t+3 of the block: codes 0,1 at k = 2t, 2t+1, codes 2,3 at
+        // k = 2t+8, 2t+9 (the queries' dims are ordered to match)
 #pragma unroll
         for (int j = 0; j < KB / 2; ++j) {
-            uint32_t w[4];   // words: (n-tile 0, k block 2j), (nt 0, 2j+1), (nt 1, 2j), (nt 1, 2j+1)
+            uint32_t w[4];
             ldsm_x4(w, st + off.k[j]);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t b0, b1;
-                fp8x4_to_f16<FMT>(w[q], b0, b1);
-                const int kk = 2 * j + (q & 1);
-                mma16816<true>(sa[q >> 1][kk % kQkChains], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
+            for (int h = 0; h < 2; ++h) {
+                uint32_t a0, a1, a2, a3;
+                fp8x4_to_f16<FMT>(w[h], a0, a2);
+                fp8x4_to_f16<FMT>(w[2 + h], a1, a3);
+                const int kk = 2 * j + h;
+                mma16816<true>(sa[kk % C], a0, a1, a2, a3, qa[kk][0], qa[kk][1]);
             }
         }
     }
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int c = 1; c < kQkChains; ++c) { sa[nt][0][0] += sa[nt][c][0]; sa[nt][0][1] += sa[nt][c][1]; }
-    // this lane: head g & 3, tokens 2t, 2t+1 (n-tile 0) and 8+2t, 9+2t (n-tile 1)
-    float s[4] = {sa[0][0][0], sa[0][0][1], sa[1][0][0], sa[1][0][1]};
+    for (int c = 1; c < C; ++c) {
+        sa[0][0] += sa[c][0]; sa[0][1] += sa[c][1]; sa[0][2] += sa[c][2]; sa[0][3] += sa[c][3];
+    }
+    float s[4] = {sa[0][0], sa[0][1], sa[0][2], sa[0][3]};
     if constexpr (FP8) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) s[e] *= skv[e];
+        s[0] *= skv[0]; s[1] *= skv[0]; s[2] *= skv[1]; s[3] *= skv[1];
     }
-    const int tA = t0 + 2 * t, tB = t0 + 8 + 2 * t;
-    const bool partial = t0 + 16 > seg_end;          // warp-uniform
-    bool v[4] = {hv, hv, hv, hv};
-    if (partial) {
-        v[0] = hv && tA < seg_end; v[1] = hv && tA + 1 < seg_end;
-        v[2] = hv && tB < seg_end; v[3] = hv && tB + 1 < seg_end;
-    }
-    if (hv && !lo) {   // raw logits for the score update, [head][slot]
-        if (!partial || tA + 1 < seg_end) *reinterpret_cast<float2*>(logit_head + tA) = make_float2(s[0], s[1]);
-        else if (tA < seg_end) logit_head[tA] = s[0];
-        if (!partial || tB + 1 < seg_end) *reinterpret_cast<float2*>(logit_head + tB) = make_float2(s[2], s[3]);
-        else if (tB < seg_end) logit_head[tB] = s[2];
+    const int tA = t0 + g, tB = t0 + 8 + g;
+    const bool inA = tA < seg_end, inB = tB < seg_end;
+    const bool v[4] = {hv0 && inA, hv1 && inA, hv0 && inB, hv1 && inB};
+    if (!lo) {   // raw logits for the score update, [head][slot]
+        float* l0 = logit_row + (size_t)(2 * t) * lstride;
+        float* l1 = l0 + lstride;
+        if (v[0]) l0[tA] = s[0];
+        if (v[1]) l1[tA] = s[1];
+        if (v[2]) l0[tB] = s[2];
+        if (v[3]) l1[tB] = s[3];
     }
 
-    // ---- online softmax with a lazy reference (moves only past 2^8)
+    // ---- online softmax with a lazy reference per head (moves only past 2^8)
     float a[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) a[e] = (s[e] - rs.m) * c2;
+    for (int e = 0; e < 4; ++e) a[e] = (s[e] - rs.m[e & 1]) * c2;
     const bool need = (v[0] && a[0] > 8.f) || (v[1] && a[1] > 8.f) || (v[2] && a[2] > 8.f) || (v[3] && a[3] > 8.f);
     if (__any_sync(kFull, need)) {
-        float mx = fmaxf(fmaxf(v[0] ? s[0] : kNegInf, v[1] ? s[1] : kNegInf),
-                         fmaxf(v[2] ? s[2] : kNegInf, v[3] ? s[3] : kNegInf));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-        const float mn = fmaxf(rs.m, mx);              // uniform over the 4 lanes of a row
-        const float al = (mn == rs.m || rs.m == kNegInf) ? (rs.m == kNegInf ? 0.f : 1.f) : ex2((rs.m - mn) * c2);
-        rs.m = mn;
-        rs.l *= al;
-        // this lane's accumulator columns 2(t & 1), 2(t & 1) + 1 hold heads 2(t & 1), +1:
-        // their factors come from the rows g = 2(t & 1), +1 (lanes 8(t & 1), 8(t & 1) + 4)
-        const float a0 = __shfl_sync(kFull, al, 8 * (t & 1)), a1 = __shfl_sync(kFull, al, 8 * (t & 1) + 4);
-        if (__any_sync(kFull, a0 != 1.f || a1 != 1.f)) {
+        float mx[2] = {fmaxf(v[0] ? s[0] : kNegInf, v[2] ? s[2] : kNegInf),
+                       fmaxf(v[1] ? s[1] : kNegInf, v[3] ? s[3] : kNegInf)};
+        float al[2];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+#pragma unroll
+            for (int m = 4; m <= 16; m <<= 1) mx[c] = fmaxf(mx[c], __shfl_xor_sync(kFull, mx[c], m));   // over tokens
+            const float mn = fmaxf(rs.m[c], mx[c]);
+            al[c] = (mn == rs.m[c] || rs.m[c] == kNegInf) ? (rs.m[c] == kNegInf ? 0.f : 1.f)
+                                                           : ex2((rs.m[c] - mn) * c2);
+            rs.m[c] = mn;
+            rs.l[c] *= al[c];
+        }
+        if (al[0] != 1.f || al[1] != 1.f) {   // this lane's accumulator columns are its two heads
 #pragma unroll
             for (int mt = 0; mt < KB; ++mt) {
-                oacc[mt][0] *= a0; oacc[mt][1] *= a1; oacc[mt][2] *= a0; oacc[mt][3] *= a1;
+                oacc[mt][0] *= al[0]; oacc[mt][1] *= al[1]; oacc[mt][2] *= al[0]; oacc[mt][3] *= al[1];
             }
         }
 #pragma unroll
-        for (int e = 0; e < 4; ++e) a[e] = (s[e] - rs.m) * c2;
+        for (int e = 0; e < 4; ++e) a[e] = (s[e] - rs.m[e & 1]) * c2;
     }
     float p[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) p[e] = v[e] ? ex2(a[e]) : 0.f;
-    rs.l += (p[0] + p[1]) + (p[2] + p[3]);
+    rs.l[0] += p[0] + p[2];
+    rs.l[1] += p[1] + p[3];
     // the accumulator holds O * vnorm: FP8 tiles fold their V scale in as well
-#pragma unroll
-    for (int e = 0; e < 4; ++e) p[e] *= FP8 ? svv[e] * vnorm : vnorm;
-    // B fragment of [P_hi | P_lo] (column g: head g & 3, high part for g < 4, low part
-    // p - hi for g >= 4) at k = 2t, 2t+1 (b0) and 2t+8, 2t+9 (b1)
-    uint32_t b0, b1;
+    const float fA = FP8 ? svv[0] * vnorm : vnorm, fB = FP8 ? svv[1] * vnorm : vnorm;
+    p[0] *= fA; p[1] *= fA; p[2] *= fB; p[3] *= fB;
+    // P rows g (tokens 0-7) and g + 8 (tokens 8-15), columns 2t, 2t + 1: high parts for
+    // t < 2, low parts p - hi for t >= 2; transposed into the B fragment (k = tokens
+    // 2t, 2t+1 in b0 and 8+2t, 9+2t in b1, n = column g)
+    uint32_t r0, r1;
     if constexpr (FP8) {
         const uint32_t h0 = pack_f16(p[0], p[1]), h1 = pack_f16(p[2], p[3]);
         const __half2 x0 = *reinterpret_cast<const __half2*>(&h0), x1 = *reinterpret_cast<const __half2*>(&h1);
-        b0 = lo ? pack_f16(p[0] - __low2float(x0), p[1] - __high2float(x0)) : h0;
-        b1 = lo ? pack_f16(p[2] - __low2float(x1), p[3] - __high2float(x1)) : h1;
+        r0 = lo ? pack_f16(p[0] - __low2float(x0), p[1] - __high2float(x0)) : h0;
+        r1 = lo ? pack_f16(p[2] - __low2float(x1), p[3] - __high2float(x1)) : h1;
     } else {
         const uint32_t h0 = pack_bf16(p[0], p[1]), h1 = pack_bf16(p[2], p[3]);
-        b0 = lo ? pack_bf16(p[0] - bf16_lo(h0), p[1] - bf16_hi(h0)) : h0;
-        b1 = lo ? pack_bf16(p[2] - bf16_lo(h1), p[3] - bf16_hi(h1)) : h1;
+        r0 = lo ? pack_bf16(p[0] - bf16_lo(h0), p[1] - bf16_hi(h0)) : h0;
+        r1 = lo ? pack_bf16(p[2] - bf16_lo(h1), p[3] - bf16_hi(h1)) : h1;
     }
+    const uint32_t b0 = movmatrix_trans(r0), b1 = movmatrix_trans(r1);
 
     // ---- O^T += V^T [P_hi | P_lo].  Past the segment end the tile holds stale slots or
     // zero fill: P is 0 there, and a partial tile also zeroes those V elements so that
     // no stale bit pattern can reach the accumulator (k = 2t, 2t+1: tokens 2t, 2t+1;
     // k = 2t+8, 2t+9: tokens 8+2t, 9+2t)
+    const int kA = t0 + 2 * t, kB = t0 + 8 + 2 * t;
+    const bool partial = t0 + 16 > seg_end;          // warp-uniform
     uint32_t m0 = 0xffffffffu, m1 = 0xffffffffu;
     if (partial) {
-        m0 = (tA < seg_end ? 0xffffu : 0u) | (tA + 1 < seg_end ? 0xffff0000u : 0u);
-        m1 = (tB < seg_end ? 0xffffu : 0u) | (tB + 1 < seg_end ? 0xffff0000u : 0u);
+        m0 = (kA < seg_end ? 0xffffu : 0u) | (kA + 1 < seg_end ? 0xffff0000u : 0u);
+        m1 = (kB < seg_end ? 0xffffu : 0u) | (kB + 1 < seg_end ? 0xffff0000u : 0u);
     }
     if (!mid()) return;
     if constexpr (!FP8) {
@@ -649,10 +675,11 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
     };
     try_issue();
 
-    const int hd = g & 3;                    // this lane's head: rows g and g + 4 repeat it
-    const bool hv = hd < d.G, lo = g >= 4;
+    // this lane's heads: columns 2t, 2t + 1 of S^T, heads (2t) & 3 and (2t + 1) & 3;
+    // lanes t >= 2 repeat those of t - 2 and supply the low parts of P
+    const bool hv0 = ((2 * t) & 3) < d.G, hv1 = ((2 * t + 1) & 3) < d.G, lo = t >= 2;
     const float c2 = (float)(p.inv_sqrt_d * 1.4426950408889634);   // log2(e) / sqrt(D)
-    RowState rs{kNegInf, 0.f};
+    RowState rs{{kNegInf, kNegInf}, {0.f, 0.f}};
     float oacc[KB][4];
 #pragma unroll
     for (int mt = 0; mt < KB; ++mt) oacc[mt][0] = oacc[mt][1] = oacc[mt][2] = oacc[mt][3] = 0.f;
@@ -711,14 +738,15 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
     if (nt16 > 0) {
         load_q<D>(sm_q, false, qa);
         const LaneOffsets<D, false> off;
-        float* logit_head = p.logit16 + ((size_t)row * 4 + (hv ? hd : 0)) * p.lstride_o;
-        const float one[4] = {1.f, 1.f, 1.f, 1.f};
+        float* logit_row = p.logit16 + (size_t)row * 4 * p.lstride_o;
+        const float one[2] = {1.f, 1.f};
         for (int i = 0; i < nt16; ++i) {
             const int t0 = 16 * (sm_tq[pos] >> 1);
             if (!wait_entry()) { aborted = true; break; }
             const uint32_t sk = ring + pos * SLOT, sv = ring + ((pos + 1) & (kSlots - 1)) * SLOT;
             bool v_ok = true;
-            attend_tile<D, false, FMT>(sk, sv, off, t0, n16, hv, lo, c2, one, one, 1.f, logit_head, qa, rs, oacc,
+            attend_tile<D, false, FMT>(sk, sv, off, t0, n16, hv0, hv1, lo, c2, one, one, 1.f, logit_row, p.lstride_o,
+                                       qa, rs, oacc,
                                        [&]() {   // K is read: free its slot, then wait for V
                                            release();
                                            v_ok = wait_entry();
@@ -732,7 +760,7 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
     if (!aborted && nt > nt16) {
         load_q<D>(sm_q, true, qa);
         const LaneOffsets<D, true> off;
-        float* logit_head = p.logit8 + ((size_t)row * 4 + (hv ? hd : 0)) * p.lstride_q;
+        float* logit_row = p.logit8 + (size_t)row * 4 * p.lstride_q;
         for (int i = nt16; i < nt; ++i) {
             const int t0 = 16 * (sm_tq[pos] >> 1);
             if (!wait_entry()) { aborted = true; break; }
@@ -744,20 +772,15 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
                 default: cp_async_wait<3>(); break;
             }
             __syncwarp();
-            // scales of this lane's tokens; zero past the segment end, where P is zero and
-            // a stale scale (NaN or Inf bits included) must not reach the product p * sv
+            // scales of this lane's tokens g and g + 8; zero past the segment end, where P
+            // is zero and a stale scale (NaN or Inf bits included) must not reach p * sv
             const float* sc = sm_sc + pos * 32;
-            float skv[4], svv[4];
-            const int tk[4] = {2 * t, 2 * t + 1, 8 + 2 * t, 9 + 2 * t};
+            const bool okA = t0 + g < n8, okB = t0 + 8 + g < n8;
+            const float skv[2] = {okA ? sc[g] : 0.f, okB ? sc[8 + g] : 0.f};
+            const float svv[2] = {okA ? sc[16 + g] : 0.f, okB ? sc[24 + g] : 0.f};
+            float m = fmaxf(svv[0], svv[1]);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const bool ok = t0 + tk[e] < n8;
-                skv[e] = ok ? sc[tk[e]] : 0.f;
-                svv[e] = ok ? sc[16 + tk[e]] : 0.f;
-            }
-            float m = fmaxf(fmaxf(svv[0], svv[1]), fmaxf(svv[2], svv[3]));
-            m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
-            m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));   // the tile's largest V scale (every lane)
+            for (int x = 4; x <= 16; x <<= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, x));   // the tile's largest V scale
             if (m > vcur) {
                 const float vn = 64.f / m, f = vn / vnorm;
 #pragma unroll
@@ -768,8 +791,8 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
                 vcur = m;
             }
             const uint32_t st = ring + pos * SLOT;
-            attend_tile<D, true, FMT>(st, st, off, t0, n8, hv, lo, c2, skv, svv, vnorm, logit_head, qa, rs, oacc,
-                                      []() { return true; });
+            attend_tile<D, true, FMT>(st, st, off, t0, n8, hv0, hv1, lo, c2, skv, svv, vnorm, logit_row, p.lstride_q,
+                                      qa, rs, oacc, []() { return true; });
             release();
         }
     }
@@ -792,13 +815,17 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
     float (*sm_l)[4] = reinterpret_cast<float (*)[4]>(smem + SL::kL);
     float (*sm_w)[4] = reinterpret_cast<float (*)[4]>(smem + SL::kRed);
     float* sm_max = reinterpret_cast<float*>(smem + SL::kMax);
-    // warp totals: l of head g over the 4 lanes of row g (rows 4..7 repeat 0..3).  o:
-    // oacc[mt] = O^T at dims 16 mt + g (c0, c1) and 16 mt + g + 8 (c2, c3), columns
-    // 2t, 2t+1; columns 0..3 hold the high part, 4..7 the low part of heads 0..3, so
-    // lanes t and t ^ 2 add up.  The accumulator carries vnorm, taken out here.
-    float l = rs.l;
-    l += __shfl_xor_sync(kFull, l, 1);
-    l += __shfl_xor_sync(kFull, l, 2);
+    // warp totals: l of heads 2t, 2t + 1 over the 8 lanes of column pair t (lanes t >= 2
+    // repeat t - 2).  o: oacc[mt] = O^T at dims 16 mt + g (c0, c1) and 16 mt + g + 8
+    // (c2, c3), columns 2t, 2t+1; columns 0..3 hold the high part, 4..7 the low part of
+    // heads 0..3, so lanes t and t ^ 2 add up.  The accumulator carries vnorm, taken out
+    // here.
+    float l0 = rs.l[0], l1 = rs.l[1];
+#pragma unroll
+    for (int x = 4; x <= 16; x <<= 1) {
+        l0 += __shfl_xor_sync(kFull, l0, x);
+        l1 += __shfl_xor_sync(kFull, l1, x);
+    }
     const float un = vcur > 0.f ? vcur * (1.f / 64.f) : 1.f;   // 1 / vnorm
 #pragma unroll
     for (int mt = 0; mt < KB; ++mt)
@@ -813,9 +840,11 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
             sm_o[warp][2 * t + 1][16 * mt + g + 8] = oacc[mt][3] * un;
         }
     }
-    if (g < 4 && t == 0) {
-        sm_l[warp][g] = l;
-        sm_m[warp][g] = rs.m;
+    if (lane < 2) {   // g = 0, t = lane: heads 2t, 2t + 1
+        sm_l[warp][2 * lane] = l0;
+        sm_l[warp][2 * lane + 1] = l1;
+        sm_m[warp][2 * lane] = rs.m[0];
+        sm_m[warp][2 * lane + 1] = rs.m[1];
     }
     __syncthreads();
     if (tid < 16) {
