@@ -623,21 +623,30 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
     const uint32_t sc_base = smem_u32(sm_sc);
     const int b = row / d.hkv, gk = row - b * d.hkv;
 
-    // this warp's tiles: list positions warp, warp + 4, ... of [bf16 tiles, FP8 tiles]
-    const int L16 = e16 - a16, L = L16 + (e8 - a8);
+    // this warp's tiles: bf16 tiles warp, warp + 4, ... of [a16, e16) and FP8 tiles
+    // warp, warp + 4, ... of [a8, e8), interleaved evenly (after i tiles, floor(i nt8 /
+    // nt) of them are FP8), so that the FP8 tiles' heavier arithmetic per byte is spread
+    // over the whole stream instead of ending it
+    const int L16 = e16 - a16, L8 = e8 - a8;
     const int nt16 = L16 > warp ? (L16 - warp + kWarps - 1) / kWarps : 0;
-    const int nt = L > warp ? (L - warp + kWarps - 1) / kWarps : 0;
-    auto enc_of = [&](int i) {   // the warp's i-th tile: (tile << 1) | fp8
-        const int li = warp + kWarps * i;
-        return li < L16 ? (a16 + li) << 1 : ((a8 + li - L16) << 1) | 1;
-    };
+    const int nt8 = L8 > warp ? (L8 - warp + kWarps - 1) / kWarps : 0;
+    const int nt = nt16 + nt8;
     // producer state (every lane keeps it; lane 0 issues the tensor loads).  The ring
     // holds entries, one slot each: a bf16 tile is two (its K, then its V), so its K slot
     // is refilled as soon as QK^T has read it; an FP8 tile is one (K and V)
     int iss = 0, half = 0, ipos = 0, free_slots = kSlots, ient = 0;
+    int berr = 0, i16 = 0, i8 = 0, enc = 0;   // the interleave (Bresenham) and the tile being issued
     auto try_issue = [&]() {
         while (iss < nt && free_slots > 0) {
-            const int enc = enc_of(iss);
+            if (half == 0) {   // the next tile: (tile << 1) | fp8
+                berr += nt8;
+                if (berr >= nt) {
+                    berr -= nt;
+                    enc = ((a8 + warp + kWarps * i8++) << 1) | 1;
+                } else {
+                    enc = (a16 + warp + kWarps * i16++) << 1;
+                }
+            }
             const bool f8 = enc & 1;
             const int jt = enc >> 1;
             const uint32_t dst = ring + ipos * SLOT, bar = bars + 8 * ipos;
@@ -732,21 +741,28 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
         try_issue();
     };
 
-    uint32_t qa[KB][2];
-    float vnorm = 1.f, vcur = 0.f;   // vcur: the largest V scale seen, 0 before any FP8 tile
-    // ---- bf16 tiles
-    if (nt16 > 0) {
-        load_q<D>(sm_q, false, qa);
-        const LaneOffsets<D, false> off;
-        float* logit_row = p.logit16 + (size_t)row * 4 * p.lstride_o;
-        const float one[2] = {1.f, 1.f};
-        for (int i = 0; i < nt16; ++i) {
-            const int t0 = 16 * (sm_tq[pos] >> 1);
-            if (!wait_entry()) { aborted = true; break; }
+    // query fragments for both kinds of tile (bf16 in natural dimension order, f16 in
+    // the FP8 words' order), held for the whole interleaved stream
+    uint32_t qa16[KB][2], qa8[KB][2];
+    if (nt16 > 0) load_q<D>(sm_q, false, qa16);
+    if (nt8 > 0) load_q<D>(sm_q, true, qa8);
+    const LaneOffsets<D, false> off16;
+    const LaneOffsets<D, true> off8;
+    float* const logit16 = p.logit16 + (size_t)row * 4 * p.lstride_o;
+    float* const logit8 = p.logit8 + (size_t)row * 4 * p.lstride_q;
+    const float one[2] = {1.f, 1.f};
+    // vcur: the largest V scale seen (0 before any FP8 tile); the accumulator holds
+    // O * vnorm, so every tile's P, bf16 tiles' included, carries the current vnorm
+    float vnorm = 1.f, vcur = 0.f;
+    for (int i = 0; i < nt; ++i) {
+        const int te = sm_tq[pos];
+        const int t0 = 16 * (te >> 1);
+        if (!wait_entry()) { aborted = true; break; }
+        if (!(te & 1)) {   // ---- a bf16 tile: its K entry, then its V entry
             const uint32_t sk = ring + pos * SLOT, sv = ring + ((pos + 1) & (kSlots - 1)) * SLOT;
             bool v_ok = true;
-            attend_tile<D, false, FMT>(sk, sv, off, t0, n16, hv0, hv1, lo, c2, one, one, 1.f, logit_row, p.lstride_o,
-                                       qa, rs, oacc,
+            attend_tile<D, false, FMT>(sk, sv, off16, t0, n16, hv0, hv1, lo, c2, one, one, vnorm, logit16,
+                                       p.lstride_o, qa16, rs, oacc,
                                        [&]() {   // K is read: free its slot, then wait for V
                                            release();
                                            v_ok = wait_entry();
@@ -754,16 +770,7 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
                                        });
             if (!v_ok) { aborted = true; break; }
             release();
-        }
-    }
-    // ---- FP8 tiles
-    if (!aborted && nt > nt16) {
-        load_q<D>(sm_q, true, qa);
-        const LaneOffsets<D, true> off;
-        float* logit_row = p.logit8 + (size_t)row * 4 * p.lstride_q;
-        for (int i = nt16; i < nt; ++i) {
-            const int t0 = 16 * (sm_tq[pos] >> 1);
-            if (!wait_entry()) { aborted = true; break; }
+        } else {           // ---- an FP8 tile: K and V in one entry, scales beside it
             // this tile's scale group (the groups of later entries may still be in flight)
             switch (ient - cent - 1) {
                 case 0: cp_async_wait<0>(); break;
@@ -791,8 +798,8 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
                 vcur = m;
             }
             const uint32_t st = ring + pos * SLOT;
-            attend_tile<D, true, FMT>(st, st, off, t0, n8, hv0, hv1, lo, c2, skv, svv, vnorm, logit_row, p.lstride_q,
-                                      qa, rs, oacc, []() { return true; });
+            attend_tile<D, true, FMT>(st, st, off8, t0, n8, hv0, hv1, lo, c2, skv, svv, vnorm, logit8, p.lstride_q,
+                                      qa8, rs, oacc, []() { return true; });
             release();
         }
     }
