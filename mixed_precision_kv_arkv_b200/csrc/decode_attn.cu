@@ -589,6 +589,42 @@ __device__ __forceinline__ Share grid_share(const AttnParams& p, char* sm) {
     return Share{out[0], out[1], out[2], out[3], out[4], out[5]};
 }
 
+// This warp's FP8 tiles among the CTA's L8: a contiguous run [*start, *start + *count).
+// The bf16 tiles are dealt round robin (warp v gets ceil((L16 - v) / 4) of them, two
+// ring entries each); the FP8 tiles (one entry each) then level the warps' entry
+// counts: first the warps one bf16 tile short, then all four evenly, so that no two
+// warps differ by more than one entry whenever L8 allows it.  Every warp computes the
+// same split, so the runs partition the L8 tiles.
+__device__ __forceinline__ void warp_fp8_share(int L16, int L8, int warp, int* start, int* count) {
+    int b[kWarps], f[kWarps];
+#pragma unroll
+    for (int v = 0; v < kWarps; ++v) b[v] = L16 > v ? 2 * ((L16 - v + kWarps - 1) / kWarps) : 0;
+    const int hi = b[0], lo = b[kWarps - 1];   // b is non-increasing, hi - lo is 0 or 2
+    int nlo = 0;
+#pragma unroll
+    for (int v = 0; v < kWarps; ++v) nlo += b[v] == lo ? 1 : 0;   // the last nlo warps
+    const int gap = (hi - lo) * nlo;
+    if (L8 <= gap) {   // only the low warps take FP8 tiles
+#pragma unroll
+        for (int v = 0; v < kWarps; ++v) {
+            const int j = v - (kWarps - nlo);
+            f[v] = j < 0 ? 0 : L8 / nlo + (j < L8 % nlo ? 1 : 0);
+        }
+    } else {
+        const int rest = L8 - gap;
+#pragma unroll
+        for (int v = 0; v < kWarps; ++v) f[v] = (b[v] == lo ? hi - lo : 0) + rest / kWarps + (v < rest % kWarps ? 1 : 0);
+    }
+    int s0 = 0, cnt = 0;   // (selects, not an indexed load: the arrays stay in registers)
+#pragma unroll
+    for (int v = 0; v < kWarps; ++v) {
+        s0 += v < warp ? f[v] : 0;
+        cnt = v == warp ? f[v] : cnt;
+    }
+    *start = s0;
+    *count = cnt;
+}
+
 // The CTA's tiles: bf16 tiles [a16, e16) then FP8 tiles [a8, e8) of its row (16
 // tokens each), dealt round robin to the warps.  Each warp streams its tiles through
 // its own ring of kSlots slots (a bf16 tile takes two, an FP8 tile one) filled by
@@ -623,13 +659,14 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
     const uint32_t sc_base = smem_u32(sm_sc);
     const int b = row / d.hkv, gk = row - b * d.hkv;
 
-    // this warp's tiles: bf16 tiles warp, warp + 4, ... of [a16, e16) and FP8 tiles
-    // warp, warp + 4, ... of [a8, e8), interleaved evenly (after i tiles, floor(i nt8 /
-    // nt) of them are FP8), so that the FP8 tiles' heavier arithmetic per byte is spread
-    // over the whole stream instead of ending it
+    // this warp's tiles: bf16 tiles warp, warp + 4, ... of [a16, e16) and its run of
+    // FP8 tiles (warp_fp8_share: the four warps stream about the same bytes),
+    // interleaved evenly (after i tiles, floor(i nt8 / nt) of them are FP8), so that
+    // the FP8 tiles' heavier arithmetic per byte is spread over the whole stream
     const int L16 = e16 - a16, L8 = e8 - a8;
     const int nt16 = L16 > warp ? (L16 - warp + kWarps - 1) / kWarps : 0;
-    const int nt8 = L8 > warp ? (L8 - warp + kWarps - 1) / kWarps : 0;
+    int f8_start, nt8;
+    warp_fp8_share(L16, L8, warp, &f8_start, &nt8);
     const int nt = nt16 + nt8;
     // producer state (every lane keeps it; lane 0 issues the tensor loads).  The ring
     // holds entries, one slot each: a bf16 tile is two (its K, then its V), so its K slot
@@ -642,7 +679,7 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
                 berr += nt8;
                 if (berr >= nt) {
                     berr -= nt;
-                    enc = ((a8 + warp + kWarps * i8++) << 1) | 1;
+                    enc = ((a8 + f8_start + i8++) << 1) | 1;
                 } else {
                     enc = (a16 + warp + kWarps * i16++) << 1;
                 }
@@ -1028,11 +1065,20 @@ __global__ void __launch_bounds__(32 * kWarps, ARKV_MIN_CTAS) decode_attn_kernel
     const int n8 = min(max(sh.n8, 0), d.cap_q);      // capacities before any use
     const bool append = n16 < d.cap_o;               // the new token goes to slot n16
     const int pos_new = p.ctx_len[row / d.hkv] + p.step;   // at this position (read at entry)
-    // this CTA's share of the row: the same fraction of each segment's 16-token tiles,
-    // so that every CTA of the row has the same mix of bf16 and FP8 work
+    // this CTA's share of the row: about the same fraction of each segment's 16-token
+    // tiles, so that every CTA of the row has about the same mix of bf16 and FP8 work.
+    // The bf16 split is floor(T16 c / n); the FP8 split is shifted by up to two tiles to
+    // even out the ring entries (two per bf16 tile, one per FP8 tile): F(c) = round(T8 c
+    // / n + 2 frac(T16 c / n)), which grows with c when T8 >= 2n (the plain split
+    // floor(T8 c / n) otherwise), with F(0) = 0 and F(n) = T8
     const int T16 = (n16 + 15) / 16, T8 = (n8 + 15) / 16;
     const int a16 = (int)((long long)T16 * sh.c / sh.n), e16 = (int)((long long)T16 * (sh.c + 1) / sh.n);
-    const int a8 = (int)((long long)T8 * sh.c / sh.n), e8 = (int)((long long)T8 * (sh.c + 1) / sh.n);
+    auto fp8_before = [&](int c) -> int {
+        const long long n = sh.n;
+        if (T8 < 2 * n) return (int)((long long)T8 * c / n);
+        return (int)((2ll * T8 * c + 4ll * (((long long)T16 * c) % n) + n) / (2 * n));
+    };
+    const int a8 = fp8_before(sh.c), e8 = fp8_before(sh.c + 1);
 
     if (e16 > a16 || e8 > a8) {
         if (lane == 0) {
