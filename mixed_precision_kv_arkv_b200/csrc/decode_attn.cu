@@ -65,6 +65,7 @@ constexpr int kWarps = 4;
 #endif
 constexpr bool kRowMultiple = ARKV_ROW_MULTIPLE != 0;
 
+
 constexpr int kSlots = 4;                  // ring slots per warp: a bf16 tile takes 2, an FP8 tile 1
 constexpr int kSpinLimit = 1 << 20;        // bounded mbarrier waits (~1 s worst case)
 constexpr int kMaxGrid = 2048;             // CTAs of one call at most (partial slots in the workspace)
@@ -83,8 +84,7 @@ struct Smem {
     static constexpr int kShare = kAbort + 16;                          // int [8] + int64 [4]: grid share
     static constexpr int kTileq = kShare + 64;                          // int [4][kSlots]: tile of each slot
     static constexpr int kSc = kTileq + kWarps * kSlots * 4;            // float [4][kSlots][32]: FP8 scales
-    static constexpr int kQ = kSc + kWarps * kSlots * 32 * 4;           // bf16 [4][D]: the group's queries
-    static constexpr int kBytes = kQ + 4 * D * 2 + 1024;                // + alignment slack
+    static constexpr int kBytes = kSc + kWarps * kSlots * 32 * 4 + 1024;   // + alignment slack
     static constexpr int kO = 0;                                        // float [4][4][D], in the idle ring
     static_assert(4 * 4 * D * 4 <= kRing, "the epilogue buffer must fit in the ring");
 };
@@ -489,22 +489,24 @@ __device__ __forceinline__ void attend_tile(uint32_t st, uint32_t sv, const Lane
     }
 }
 
-// A fragments (a0, a2 of every k block) of query row g: head g & 3 (rows 0..3 and
-// 4..7 repeat the group; the rows of heads >= G are zero in qs): bf16 in natural
-// dimension order; f16 for FP8 tiles, in the order of the 4-byte K words (dims
-// 16 kk + 4t .. + 3).  qs: the group's queries in shared memory, [4][D] bf16.
+// Query fragments of column g of Q^T (the B operand of S^T = K Q^T: b0, b1 of every k
+// block): head g & 3 (columns 0..3 and 4..7 repeat the group; heads >= G give zero):
+// bf16 in natural dimension order; f16 for FP8 tiles, in the order of the 4-byte K
+// words (dims 16 kk + 4t .. + 3).  qs: the group's queries in global memory, [G][D]
+// bf16, read directly by every lane (an L2 hit after the prefetch).
 template <int D>
-__device__ __forceinline__ void load_q(const uint16_t* qs, bool fp8, uint32_t (&qa)[D / 16][2]) {
+__device__ __forceinline__ void load_q(const uint16_t* qs, bool fp8, int G, uint32_t (&qa)[D / 16][2]) {
     const int lane = threadIdx.x & 31, h = (lane >> 2) & 3, t = lane & 3;
-    const uint16_t* qrow = qs + h * D;
+    const bool ok = h < G;   // rows of heads >= G are zero
+    const uint16_t* qrow = qs + (ok ? h : 0) * D;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t x, y;
+        uint32_t x = 0u, y = 0u;
         if (fp8) {
-            const uint2 u = *reinterpret_cast<const uint2*>(qrow + 16 * kk + 4 * t);
+            const uint2 u = ok ? *reinterpret_cast<const uint2*>(qrow + 16 * kk + 4 * t) : make_uint2(0u, 0u);
             x = pack_f16(bf16_lo(u.x), bf16_hi(u.x));
             y = pack_f16(bf16_lo(u.y), bf16_hi(u.y));
-        } else {
+        } else if (ok) {
             x = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * t);
             y = *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * t + 8);
         }
@@ -655,7 +657,6 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
     int* sm_abort = reinterpret_cast<int*>(smem + SL::kAbort);
     int* sm_tq = reinterpret_cast<int*>(smem + SL::kTileq) + warp * kSlots;      // (tile << 1) | fp8, by slot
     float* sm_sc = reinterpret_cast<float*>(smem + SL::kSc) + warp * kSlots * 32;  // scales, by slot
-    uint16_t* sm_q = reinterpret_cast<uint16_t*>(smem + SL::kQ);                  // [4][D] bf16
     const uint32_t sc_base = smem_u32(sm_sc);
     const int b = row / d.hkv, gk = row - b * d.hkv;
 
@@ -741,13 +742,6 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
         }
         pdl_wait();
     }
-    for (int i = tid; i < 4 * D / 8; i += blockDim.x) {   // the group's queries, zero past G
-        const int h = i / (D / 8), c = i - h * (D / 8);
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (h < d.G) v = *reinterpret_cast<const uint4*>(p.q + ((size_t)b * d.hq + gk * d.G + h) * D + 8 * c);
-        *reinterpret_cast<uint4*>(sm_q + h * D + 8 * c) = v;
-    }
-    __syncthreads();
 
     int pos = 0;          // ring slot of the next entry to consume
     uint32_t ph = 0;      // parity of every slot's next phase
@@ -781,8 +775,11 @@ __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int ro
     // query fragments for both kinds of tile (bf16 in natural dimension order, f16 in
     // the FP8 words' order), held for the whole interleaved stream
     uint32_t qa16[KB][2], qa8[KB][2];
-    if (nt16 > 0) load_q<D>(sm_q, false, qa16);
-    if (nt8 > 0) load_q<D>(sm_q, true, qa8);
+    // (each warp loads its own fragments from global memory, an L2 hit after the
+    // prefetch: no staging through shared memory and no block barrier before the stream)
+    const uint16_t* qg = p.q + ((size_t)b * d.hq + gk * d.G) * D;   // the group's queries
+    if (nt16 > 0) load_q<D>(qg, false, d.G, qa16);
+    if (nt8 > 0) load_q<D>(qg, true, d.G, qa8);
     const LaneOffsets<D, false> off16;
     const LaneOffsets<D, true> off8;
     float* const logit16 = p.logit16 + (size_t)row * 4 * p.lstride_o;
