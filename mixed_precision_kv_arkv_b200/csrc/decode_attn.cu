@@ -3,41 +3,45 @@
 // originals) and the score observation that feeds §2.나.
 //
 // One wave of CTAs (as many as the GPU holds at once) shares the rows in
-// proportion to their lengths; each CTA takes the same fraction of its row's bf16
-// tiles and of its FP8 tiles (16 tokens each), bf16 tiles first.  Its 4 warps take
-// the tiles round robin, each through its own ring of 4 shared-memory slots (a bf16
-// tile takes two, K and V, each freed as soon as it is read; an FP8 tile one) filled
-// by TMA tensor loads (16 rows per box, 128-byte swizzle; 64-byte for FP8 rows of 64
-// bytes) completing on per-slot mbarriers (waits are bounded).
+// proportion to their lengths; each CTA takes about the same fraction of its row's
+// bf16 tiles and of its FP8 tiles (16 tokens each; the FP8 split is shifted so that
+// the CTAs' ring entries match).  Its 4 warps each take bf16 tiles round robin and
+// one run of FP8 tiles (sized so that the warps' entries match), interleaved evenly,
+// each warp through its own ring of 4 shared-memory slots (a bf16 tile takes two, K
+// and V, each freed as soon as it is read; an FP8 tile one) filled by TMA tensor
+// loads (16 rows per box, 128-byte swizzle; 64-byte for FP8 rows of 64 bytes)
+// completing on per-slot mbarriers (waits are bounded).
 //
-// Tile math on the warp-level tensor cores (m16n8k16).  QK^T with the queries as
-// the M rows: rows 0..3 and 4..7 both hold the group's heads (zero past G), rows
-// 8..15 are zero, so lane (g, t) finds the logits of head g & 3 for tokens 2t,
-// 2t+1 (n-tile 0) and 8+2t, 9+2t (n-tile 1) -- exactly the entries of the B
-// fragment of [P_hi | P_lo] that it supplies for column g of
+// Tile math on the warp-level tensor cores (m16n8k16).  S^T = K Q^T: K is the A
+// operand (16 tokens of a k block per mma), the queries the B operand (column n =
+// head n & 3, zero past G), so lane (g, t) finds the logits of tokens g and g + 8
+// for heads 2t, 2t + 1 (lanes t >= 2 repeat t - 2).  Two register transposes
+// (movmatrix) turn its probabilities into the B fragment of
 //   O^T[D x 8] += V^T[D x 16 tok] * [P_hi | P_lo][16 tok x 8]
 // (columns 0..3: the 16-bit high part of each head's probabilities, 4..7 the low
-// part p - hi, so one mma carries ~16 significant bits of every probability).  P
-// never leaves the registers; hi and lo meet once at the end (lanes t, t ^ 2).
+// part p - hi, so one mma carries ~16 significant bits of every probability); a
+// lane's accumulator columns are its own heads, and hi and lo meet once at the end
+// (lanes t, t ^ 2).
 //   bf16 tiles: K fragments by ldmatrix, V^T fragments by ldmatrix.trans.
 //   FP8 tiles: codes are converted to f16 in registers (exact; E5M2 is the high
 //   byte of an f16, E4M3 goes through the hardware conversion).  K: each 4-byte
-//   word a lane reads (dims 4t..4t+3 of a 16-dim chunk) is its B fragment for that
-//   k block, and the query is loaded with the same dimension order; V: the 8-bit
-//   transposing ldmatrix gives lane (g, t) the four rows its address lanes
-//   4t..4t+3 supplied, and the rows are supplied in the token order 0,1,8,9,
-//   2,3,10,11, ... so that they are tokens 2t, 2t+1, 8+2t, 9+2t -- the k positions
-//   of the bf16 path.  The per-token K scale multiplies the finished logit; the V
-//   scale is folded into P, and P is multiplied by 64 / (the largest V scale of
-//   the warp's FP8 tiles so far; the accumulator is rescaled when it grows), which
-//   keeps p * sv inside f16 and comes back out of the partial.
-// Softmax in float32 with a reference maximum that moves only when a logit
-// exceeds it by 2^8 (so most tiles need no reduction, which is two shuffles over
-// the 4 lanes of a row when it happens).  Raw logits go to the workspace for the
-// score update.  The CTA combines its warps into one (max, sum, unnormalised o)
-// partial; the last CTA of a row to finish (a ticket in the workspace) merges the
-// row's partials and the new token into o and each head's final (max, sum), stores
-// the new token in the cache and advances the row's bf16 count past it.
+//   word a lane reads (dims 4t..4t+3 of a 16-dim chunk of one token) is its A
+//   fragment pair for that k block, and the query is loaded with the same
+//   dimension order; V: the 8-bit transposing ldmatrix gives lane (g, t) the four
+//   rows its address lanes 4t..4t+3 supplied, and the rows are supplied in the
+//   token order 0,1,8,9, 2,3,10,11, ... so that they are tokens 2t, 2t+1, 8+2t,
+//   9+2t -- the k positions of the bf16 path.  The per-token K scale multiplies the
+//   finished logit; the V scale is folded into P, and every P is multiplied by 64 /
+//   (the largest V scale of the warp's FP8 tiles so far; the accumulator is
+//   rescaled when it grows), which keeps p * sv inside f16 and comes back out of
+//   the partial.
+// Softmax in float32 with a reference maximum per head that moves only when a logit
+// exceeds it by 2^8 (so most tiles need no reduction, which is three shuffles over
+// the 8 token lanes when it happens).  Raw logits go to the workspace for the score
+// update.  The CTA combines its warps into one (max, sum, unnormalised o) partial;
+// the last CTA of a row to finish (a ticket in the workspace) merges the row's
+// partials and the new token into o and each head's final (max, sum), stores the
+// new token in the cache and advances the row's bf16 count past it.
 #include <math.h>
 #include <mutex>
 
@@ -627,8 +631,9 @@ __device__ __forceinline__ void warp_fp8_share(int L16, int L8, int warp, int* s
     *count = cnt;
 }
 
-// The CTA's tiles: bf16 tiles [a16, e16) then FP8 tiles [a8, e8) of its row (16
-// tokens each), dealt round robin to the warps.  Each warp streams its tiles through
+// The CTA's tiles: bf16 tiles [a16, e16) and FP8 tiles [a8, e8) of its row (16
+// tokens each), shared among the warps as described at the tile list below.  Each
+// warp streams its tiles, the two kinds interleaved, through
 // its own ring of kSlots slots (a bf16 tile takes two, an FP8 tile one) filled by
 // TMA; an FP8 tile's 16 K and 16 V scales come with it, one 4-byte cp.async per lane
 // into the slot's scale area (one cp.async group per issued tile).  The CTA then
@@ -642,7 +647,9 @@ __device__ __forceinline__ void warp_fp8_share(int L16, int L8, int warp, int* s
 // The V scale is folded into P in f16, so P is also multiplied by vnorm = 64 / (the
 // largest V scale among the warp's FP8 tiles so far): p sv vnorm <= 2^8 * 64 stays
 // inside f16 and well above its subnormals.  vnorm starts at 1 and the accumulator
-// is rescaled when an FP8 tile raises the maximum; it comes back out of the partial.
+// is rescaled when an FP8 tile raises the maximum; since the accumulator holds
+// O * vnorm, bf16 tiles multiply their P by the current vnorm too.  It comes back
+// out of the partial.
 template <int D, int FMT>
 __device__ __forceinline__ void cta_body(const AttnParams& p, char* smem, int row, int n16, int n8, int a16,
                                          int e16, int a8, int e8) {
