@@ -496,7 +496,10 @@ def run_arkv(args, wl, rank, world, local_rank):
 
         # the host transfers go through arkv_copy_async (a kernel reading and writing the
         # page-locked buffers), so the captured step has no copy-engine node between its
-        # kernels; one call per buffer before the capture checks each buffer
+        # kernels; one call per buffer before the capture checks each buffer.  One copy per
+        # buffer and direction per step, on the main stream: per-layer copies on side
+        # streams were slower, because the attention calls then wait on events between
+        # them and lose their programmatic early launch
         def transfers(i):
             st = torch.cuda.current_stream().cuda_stream
             for dd, hh in ((qd, qh[i]), (kd, kh[i]), (vd, vh[i])):
@@ -560,6 +563,9 @@ def run_arkv(args, wl, rank, world, local_rank):
     with ClockSampler(local_rank) as clk:
         ms_value = timed(g_value)
         ms_e2e = timed(g_e2e) if not args.no_e2e else None
+        # the last step's outputs, as copied to host memory, against the device buffer
+        # they were copied from (no pass has written it since)
+        e2e_copied = bool(torch.equal(oh[K - 1], o.cpu())) if not args.no_e2e else None
         timed(g_k)
         join()
         saved = [(x["cache"].n_bf16.clone(), x["cache"].n_fp8.clone()) for x in layers]
@@ -619,7 +625,10 @@ def run_arkv(args, wl, rank, world, local_rank):
     if not args.no_e2e:
         line["e2e"] = {"value": job_tokens_per_s(B, K, world, ms_e2e), "unit": "tokens/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                       "ms_per_step": ms_e2e / K}
+                       "ms_per_step": ms_e2e / K,
+                       "transfers": "arkv_copy_async, one per buffer and direction per step, on the "
+                                    "attention stream",
+                       "outputs_copied": e2e_copied}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_from_state(wl, layers[0], ctx_np, total_steps, o, args.cpu_seconds,
                                                        lambda t: (layer_step(0, t), join()))
