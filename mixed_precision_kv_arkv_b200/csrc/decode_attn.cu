@@ -48,6 +48,7 @@
 #include <cudaTypedefs.h>
 
 #include "arkv_internal.cuh"
+#include "splits.h"
 
 namespace arkv {
 
@@ -64,6 +65,7 @@ constexpr unsigned kFull = 0xffffffffu;
 #endif
 constexpr int kQkChains = ARKV_QK_CHAINS;   // independent QK^T accumulator chains per tile
 constexpr int kWarps = 4;
+static_assert(kWarps == kSplitWarps, "the tile splits assume the decode CTA's warp count");
 #ifndef ARKV_ROW_MULTIPLE
 #define ARKV_ROW_MULTIPLE 1
 #endif
@@ -595,42 +597,6 @@ __device__ __forceinline__ Share grid_share(const AttnParams& p, char* sm) {
     return Share{out[0], out[1], out[2], out[3], out[4], out[5]};
 }
 
-// This warp's FP8 tiles among the CTA's L8: a contiguous run [*start, *start + *count).
-// The bf16 tiles are dealt round robin (warp v gets ceil((L16 - v) / 4) of them, two
-// ring entries each); the FP8 tiles (one entry each) then level the warps' entry
-// counts: first the warps one bf16 tile short, then all four evenly, so that no two
-// warps differ by more than one entry whenever L8 allows it.  Every warp computes the
-// same split, so the runs partition the L8 tiles.
-__device__ __forceinline__ void warp_fp8_share(int L16, int L8, int warp, int* start, int* count) {
-    int b[kWarps], f[kWarps];
-#pragma unroll
-    for (int v = 0; v < kWarps; ++v) b[v] = L16 > v ? 2 * ((L16 - v + kWarps - 1) / kWarps) : 0;
-    const int hi = b[0], lo = b[kWarps - 1];   // b is non-increasing, hi - lo is 0 or 2
-    int nlo = 0;
-#pragma unroll
-    for (int v = 0; v < kWarps; ++v) nlo += b[v] == lo ? 1 : 0;   // the last nlo warps
-    const int gap = (hi - lo) * nlo;
-    if (L8 <= gap) {   // only the low warps take FP8 tiles
-#pragma unroll
-        for (int v = 0; v < kWarps; ++v) {
-            const int j = v - (kWarps - nlo);
-            f[v] = j < 0 ? 0 : L8 / nlo + (j < L8 % nlo ? 1 : 0);
-        }
-    } else {
-        const int rest = L8 - gap;
-#pragma unroll
-        for (int v = 0; v < kWarps; ++v) f[v] = (b[v] == lo ? hi - lo : 0) + rest / kWarps + (v < rest % kWarps ? 1 : 0);
-    }
-    int s0 = 0, cnt = 0;   // (selects, not an indexed load: the arrays stay in registers)
-#pragma unroll
-    for (int v = 0; v < kWarps; ++v) {
-        s0 += v < warp ? f[v] : 0;
-        cnt = v == warp ? f[v] : cnt;
-    }
-    *start = s0;
-    *count = cnt;
-}
-
 // The CTA's tiles: bf16 tiles [a16, e16) and FP8 tiles [a8, e8) of its row (16
 // tokens each), shared among the warps as described at the tile list below.  Each
 // warp streams its tiles, the two kinds interleaved, through
@@ -1076,19 +1042,11 @@ __global__ void __launch_bounds__(32 * kWarps, ARKV_MIN_CTAS) decode_attn_kernel
     const bool append = n16 < d.cap_o;               // the new token goes to slot n16
     const int pos_new = p.ctx_len[row / d.hkv] + p.step;   // at this position (read at entry)
     // this CTA's share of the row: about the same fraction of each segment's 16-token
-    // tiles, so that every CTA of the row has about the same mix of bf16 and FP8 work.
-    // The bf16 split is floor(T16 c / n); the FP8 split is shifted by up to two tiles to
-    // even out the ring entries (two per bf16 tile, one per FP8 tile): F(c) = round(T8 c
-    // / n + 2 frac(T16 c / n)), which grows with c when T8 >= 2n (the plain split
-    // floor(T8 c / n) otherwise), with F(0) = 0 and F(n) = T8
+    // tiles, so that every CTA of the row has about the same mix of bf16 and FP8 work
+    // (the FP8 split evens out the ring entries: fp8_tiles_before)
     const int T16 = (n16 + 15) / 16, T8 = (n8 + 15) / 16;
     const int a16 = (int)((long long)T16 * sh.c / sh.n), e16 = (int)((long long)T16 * (sh.c + 1) / sh.n);
-    auto fp8_before = [&](int c) -> int {
-        const long long n = sh.n;
-        if (T8 < 2 * n) return (int)((long long)T8 * c / n);
-        return (int)((2ll * T8 * c + 4ll * (((long long)T16 * c) % n) + n) / (2 * n));
-    };
-    const int a8 = fp8_before(sh.c), e8 = fp8_before(sh.c + 1);
+    const int a8 = fp8_tiles_before(T16, T8, sh.n, sh.c), e8 = fp8_tiles_before(T16, T8, sh.n, sh.c + 1);
 
     if (e16 > a16 || e8 > a8) {
         if (lane == 0) {
